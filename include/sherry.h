@@ -1,0 +1,175 @@
+/*
+ * sherry.h -- C ABI of libsherry_b200.so: the Sherry 3:4 ternary-weight matmul
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method (Sherry page, pnsm.cn/news/1195499, "Sherry framework: ternary
+ * quantisation and 3:4 sparsity for LLM inference"):
+ *   - sec. 3.1: every group of 4 consecutive weights along K is replaced by
+ *     T in {-1,0,+1}^4 with exactly 3 nonzeros -- the 3 largest |w| keep
+ *     their signs -- times a least-squares scale alpha (one per output row n);
+ *   - sec. 2.1: each group is stored as one 5-bit code (1.25 bit/weight);
+ *   - sec. 2.2: activations are integers, the contraction is additions and
+ *     subtractions accumulated exactly, followed by float scaling.
+ *
+ * Data conventions (all row-major):
+ *   W      fp32 [N][K]      output feature n is row n (Linear.weight layout)
+ *   x      fp32 [M][K]      M tokens
+ *   x_i8   int8 [M][K]      quantised activations, x_scale fp32 [M]
+ *   y      fp32 [M][N]      y[m][n] = (float)((float)acc[m][n] * alpha[n]) * x_scale[m]
+ *   acc    int32 [M][N]     acc[m][n] = sum_k x_i8[m][k] * T[n][k]  (exact)
+ *
+ * Canonical code of a group (z = position of the zero, s_j = 1 when the j-th
+ * kept weight in ascending position is negative):
+ *     code = z | s0 << 2 | s1 << 3 | s2 << 4
+ * Canonical stream: row n starts at byte n * (5K/32); code g occupies stream
+ * bits [5g, 5g+5), least significant bit first (bit b is bit b%8 of byte b/8).
+ *
+ * Shape rules: M, N, K >= 1 and K % 32 == 0 (rows of whole bytes).
+ *
+ * Ownership: the caller owns every buffer passed in.  Host functions take host
+ * pointers; device functions take device pointers and a cudaStream_t passed
+ * as void* (NULL = legacy default stream).  Device functions are asynchronous
+ * on that stream; none of them synchronises.  The only device memory the
+ * library allocates itself is one workspace per device for split-K partial
+ * sums, created on the first sherry_gemm call that needs it, grown when a
+ * larger problem arrives, and kept (all zero between calls) until exit.
+ *
+ * Errors: every function returns a sherry_status.  Argument errors are
+ * reported before anything is launched.  SHERRY_ERR_CUDA means a CUDA call
+ * (launch, copy, allocation) failed; the CUDA error is then also left for
+ * cudaGetLastError.  Kernels never trap: a wait that exceeds its bound sets a
+ * device status word (read with sherry_last_device_status) and the kernel
+ * returns.
+ */
+#ifndef SHERRY_H
+#define SHERRY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SHERRY_OK = 0,
+    SHERRY_ERR_INVALID_ARG = 1,       /* null pointer, non-positive size, misaligned pointer */
+    SHERRY_ERR_UNSUPPORTED_SHAPE = 2, /* K % 32 != 0, or a size beyond the int32 index range */
+    SHERRY_ERR_NONFINITE = 3,         /* NaN or Inf in W (sherry_pack) */
+    SHERRY_ERR_CUDA = 4,              /* a CUDA runtime call failed */
+    SHERRY_ERR_DEVICE = 5             /* the device is not sm_100 or lacks a needed feature */
+} sherry_status;
+
+/* Short English text for a status value; never NULL. */
+const char* sherry_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int sherry_version(void);
+
+/* Bytes of the canonical code stream for an N x K weight: N * K * 5 / 32
+ * (sec. 2.1, 1.25 bit/weight).  Returns 0 for invalid shapes. */
+size_t sherry_packed_bytes(int64_t N, int64_t K);
+
+/* Bytes of the kernel-native layout written by sherry_repack and read by
+ * sherry_gemm: rows padded to a multiple of 128 and K to a multiple of 128,
+ * 20 bytes per (row, 128-wide K chunk).  Returns 0 for invalid shapes. */
+size_t sherry_native_bytes(int64_t N, int64_t K);
+
+/*
+ * sherry_pack -- host, synchronous.  Offline ternarisation and packing
+ * (sec. 3.1 objective, sec. 2.1 encoding).
+ *   W      [in]  fp32 [N][K], host memory, finite values only
+ *   codes  [out] uint8 [N][5K/32], host memory (canonical stream)
+ *   alpha  [out] fp32 [N], host memory: sum of kept |w| (fp64, ascending k)
+ *                / (0.75 K), rounded once to fp32
+ * Per group the smallest |w| is zeroed (lowest index on ties); kept weights
+ * keep their sign (w < 0 is negative, so -0.0 counts as +).
+ * Returns SHERRY_ERR_NONFINITE (outputs unspecified) if W holds NaN or Inf.
+ * Uses the host's cores (OpenMP over rows); results do not depend on the
+ * number of threads.
+ */
+int sherry_pack(const float* W, int64_t N, int64_t K, uint8_t* codes, float* alpha);
+
+/*
+ * sherry_unpack -- host, synchronous.  Canonical codes -> T int8 [N][K] in
+ * {-1,0,+1} (exactly 3 nonzeros per group).  Every 5-bit value is a valid
+ * code, so any byte stream decodes.
+ */
+int sherry_unpack(const uint8_t* codes, int64_t N, int64_t K, int8_t* T);
+
+/*
+ * sherry_repack -- device, asynchronous on `stream`.  Rearranges a canonical
+ * code stream already copied to the device into the kernel-native layout
+ * (same codes, tile-interleaved so that 128 consecutive rows of one 128-wide
+ * K chunk are one contiguous 2560-byte block).
+ *   codes_dev  [in]  uint8 [N][5K/32], device memory
+ *   native_dev [out] sherry_native_bytes(N, K) bytes, device memory, 16-byte aligned
+ * Padding bytes are written as zero.
+ */
+int sherry_repack(const uint8_t* codes_dev, int64_t N, int64_t K, void* native_dev,
+                  void* stream);
+
+/*
+ * sherry_quant_act -- device, asynchronous.  Per-token int8 activation
+ * quantisation (sec. 2.2 step 1 leaves the rule open; this is symmetric
+ * absmax/127 with round-half-to-even and IEEE fp32 division):
+ *   a = max_k |x[m][k]|;  x_scale[m] = a / 127;
+ *   x_i8[m][k] = clamp(rint(x[m][k] / x_scale[m]), -127, 127);
+ *   a == 0 gives x_scale[m] = 0 and a zero row.
+ *   x       [in]  fp32 [M][K], device memory, 16-byte aligned
+ *   x_i8    [out] int8 [M][K], device memory, 16-byte aligned
+ *   x_scale [out] fp32 [M], device memory
+ * NaN or Inf in x gives unspecified values (no error is reported).
+ */
+int sherry_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_i8, float* x_scale,
+                     void* stream);
+
+/*
+ * sherry_gemm -- device, asynchronous.  y = epilogue(x_i8 . T^T) (sec. 2.2
+ * steps 2-4): exact int32 accumulation on the tensor cores (tcgen05 kind::i8,
+ * ternary weights decoded from the 5-bit codes into tensor memory), then
+ * y[m][n] = (float)((float)acc * alpha[n]) * x_scale[m].
+ *   x_i8     [in]  int8 [M][K], device memory, 16-byte aligned
+ *   x_scale  [in]  fp32 [M], device memory
+ *   Wnative  [in]  kernel-native codes from sherry_repack, device memory, 16-byte aligned
+ *   alpha    [in]  fp32 [N], device memory
+ *   y        [out] fp32 [M][N], device memory
+ * Calls on the same device share the split-K workspace: calls that may run
+ * at the same time on different streams must not be issued (serialise them
+ * on one stream or with events).
+ */
+int sherry_gemm(const int8_t* x_i8, const float* x_scale, const void* Wnative,
+                const float* alpha, float* y, int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * sherry_gemm_acc -- as sherry_gemm, and also writes the exact int32
+ * accumulators acc[M][N] (device memory) when acc != NULL.  y may be NULL
+ * when only acc is wanted.
+ */
+int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnative,
+                    const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,
+                    int64_t K, void* stream);
+
+/*
+ * sherry_gemm_simt -- device, asynchronous.  The same contraction and
+ * epilogue on the CUDA cores (shared-memory code table + dp4a), kept as an
+ * independent second kernel for A/B comparison.  Same arguments as
+ * sherry_gemm_acc; needs no workspace.
+ */
+int sherry_gemm_simt(const int8_t* x_i8, const float* x_scale, const void* Wnative,
+                     const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,
+                     int64_t K, void* stream);
+
+/*
+ * sherry_last_device_status -- host, synchronous (copies one word from the
+ * current device).  0 when no kernel of this library has reported a bounded
+ * wait running out since the last reset; otherwise a nonzero code naming the
+ * wait.  reset != 0 clears it.
+ */
+int sherry_last_device_status(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SHERRY_H */

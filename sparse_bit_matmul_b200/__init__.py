@@ -1,0 +1,198 @@
+"""Python binding of libsherry_b200 (include/sherry.h): the Sherry 3:4 ternary
+matmul on B200.
+
+Only argument marshalling lives here: every step of the path runs in the C /
+CUDA library.  Host functions take numpy arrays; device functions take torch
+CUDA tensors (torch supplies device memory and the current stream).  There
+is no fallback: if the library is missing or a call fails, an exception is
+raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SO_PATH = os.path.join(HERE, "libsherry_b200.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_NONFINITE, ERR_CUDA, ERR_DEVICE = range(6)
+
+# every entry point declared in include/sherry.h
+ABI_SYMBOLS = (
+    "sherry_status_string", "sherry_version", "sherry_packed_bytes", "sherry_native_bytes",
+    "sherry_pack", "sherry_unpack", "sherry_repack", "sherry_quant_act", "sherry_gemm",
+    "sherry_gemm_acc", "sherry_gemm_simt", "sherry_last_device_status",
+)
+
+_lib = None
+
+
+class SherryError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree library; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(SO_PATH):
+        raise ImportError(f"{SO_PATH} is missing: run `python -m sparse_bit_matmul_b200.build`")
+    L = ctypes.CDLL(SO_PATH)
+    i64, vp, c_int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+    L.sherry_status_string.argtypes = [c_int]
+    L.sherry_status_string.restype = ctypes.c_char_p
+    L.sherry_version.restype = c_int
+    L.sherry_packed_bytes.argtypes = [i64, i64]
+    L.sherry_packed_bytes.restype = ctypes.c_size_t
+    L.sherry_native_bytes.argtypes = [i64, i64]
+    L.sherry_native_bytes.restype = ctypes.c_size_t
+    L.sherry_pack.argtypes = [vp, i64, i64, vp, vp]
+    L.sherry_unpack.argtypes = [vp, i64, i64, vp]
+    L.sherry_repack.argtypes = [vp, i64, i64, vp, vp]
+    L.sherry_quant_act.argtypes = [vp, i64, i64, vp, vp, vp]
+    L.sherry_gemm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_gemm_acc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_gemm_simt.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_last_device_status.argtypes = [c_int]
+    for name in ABI_SYMBOLS:
+        getattr(L, name).restype = getattr(L, name).restype or c_int
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return load().sherry_status_string(int(status)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise SherryError(what, rc)
+
+
+def _np_ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _dptr(t):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "device arguments must be contiguous CUDA tensors"
+    return t.data_ptr()
+
+
+def _stream(t):
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+# ----------------------------------------------------------------- host side
+def packed_bytes(N: int, K: int) -> int:
+    return int(load().sherry_packed_bytes(N, K))
+
+
+def native_bytes(N: int, K: int) -> int:
+    return int(load().sherry_native_bytes(N, K))
+
+
+def pack(W: np.ndarray):
+    """fp32 W [N][K] -> (canonical codes uint8 [N][5K/32], alpha fp32 [N])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    codes = np.empty((N, K // 32 * 5), dtype=np.uint8)
+    alpha = np.empty(N, dtype=np.float32)
+    _check(load().sherry_pack(_np_ptr(W), N, K, _np_ptr(codes), _np_ptr(alpha)), "sherry_pack")
+    return codes, alpha
+
+
+def unpack(codes: np.ndarray, K: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    N = codes.shape[0]
+    T = np.empty((N, K), dtype=np.int8)
+    _check(load().sherry_unpack(_np_ptr(codes), N, K, _np_ptr(T)), "sherry_unpack")
+    return T
+
+
+# --------------------------------------------------------------- device side
+def repack(codes_dev, N: int, K: int, out=None):
+    """Canonical codes on the device -> kernel-native layout (uint8 tensor)."""
+    import torch
+    if out is None:
+        out = torch.empty(native_bytes(N, K), dtype=torch.uint8, device=codes_dev.device)
+    _check(load().sherry_repack(_dptr(codes_dev), N, K, _dptr(out), _stream(codes_dev)), "sherry_repack")
+    return out
+
+
+def quant_act(x, out_q=None, out_s=None):
+    """fp32 x [M][K] -> (int8 [M][K], fp32 scale [M])."""
+    import torch
+    M, K = x.shape
+    q = out_q if out_q is not None else torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s = out_s if out_s is not None else torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(load().sherry_quant_act(_dptr(x), M, K, _dptr(q), _dptr(s), _stream(x)), "sherry_quant_act")
+    return q, s
+
+
+def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: bool = True,
+         kernel: str = "tc"):
+    """y fp32 [M][N] (and optionally exact int32 acc) from int8 activations and
+    kernel-native codes.  kernel="simt" runs the CUDA-core comparison kernel."""
+    import torch
+    M, K = x_i8.shape
+    y = None
+    if want_y:
+        y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x_i8.device)
+    L = load()
+    args = (_dptr(x_i8), _dptr(x_scale), _dptr(w_native), _dptr(alpha), _dptr(y), _dptr(acc), M, N, K,
+            _stream(x_i8))
+    if kernel == "tc":
+        if acc is None:
+            rc = L.sherry_gemm(args[0], args[1], args[2], args[3], args[4], M, N, K, args[-1])
+        else:
+            rc = L.sherry_gemm_acc(*args)
+    elif kernel == "simt":
+        rc = L.sherry_gemm_simt(*args)
+    else:
+        raise ValueError(kernel)
+    _check(rc, f"sherry_gemm[{kernel}]")
+    return y
+
+
+def last_device_status(reset: bool = False) -> int:
+    return int(load().sherry_last_device_status(1 if reset else 0))
+
+
+class PackedLinear:
+    """Weights of one Sherry linear layer resident on the device.
+
+    ``PackedLinear.from_weights(W)`` packs on the host (sherry_pack), copies
+    the canonical codes and alpha to the device and repacks them into the
+    kernel-native layout.  ``forward(x)`` quantises the activations and runs
+    the GEMM; both are asynchronous on the current stream.
+    """
+
+    def __init__(self, w_native, alpha, N: int, K: int):
+        self.w_native, self.alpha, self.N, self.K = w_native, alpha, N, K
+
+    @classmethod
+    def from_weights(cls, W: np.ndarray, device="cuda"):
+        import torch
+        codes, alpha = pack(W)
+        return cls.from_codes(codes, alpha, W.shape[1], device)
+
+    @classmethod
+    def from_codes(cls, codes: np.ndarray, alpha: np.ndarray, K: int, device="cuda"):
+        import torch
+        N = codes.shape[0]
+        codes_d = torch.from_numpy(codes).to(device)
+        w_native = repack(codes_d, N, K)
+        return cls(w_native, torch.from_numpy(alpha).to(device), N, K)
+
+    def forward(self, x, out=None):
+        q, s = quant_act(x)
+        return gemm(q, s, self.w_native, self.alpha, self.N, out=out)

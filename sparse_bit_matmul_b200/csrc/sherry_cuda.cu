@@ -1,0 +1,397 @@
+// Device half of libsherry_b200: activation quantiser, repack, the SIMT
+// comparison kernel, the tcgen05 GEMM launcher and the device entry points of
+// the C ABI (include/sherry.h).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "sherry.h"
+#include "sherry_internal.h"
+#include "tc_gemm.cuh"
+
+namespace sherry {
+
+__device__ unsigned g_device_status = 0;
+
+// ---------------------------------------------------------------------------
+// Activation quantiser: one CTA per token.  a = max |x| (exact), s = a / 127
+// (IEEE fp32 division), q = clamp(rint(x / s), -127, 127) with rint rounding
+// half to even; a == 0 gives s = 0 and q = 0.
+// ---------------------------------------------------------------------------
+constexpr int kQuantThreads = 256;
+
+__global__ void __launch_bounds__(kQuantThreads)
+    quant_act_kernel(const float* __restrict__ x, int64_t K, int8_t* __restrict__ q, float* __restrict__ scale)
+{
+    const int64_t m = blockIdx.x;
+    const float4* xr = reinterpret_cast<const float4*>(x + m * K);
+    char4* qr = reinterpret_cast<char4*>(q + m * K);
+    const int64_t K4 = K / 4;
+
+    float a = 0.0f;
+    for (int64_t i = threadIdx.x; i < K4; i += kQuantThreads) {
+        const float4 v = xr[i];
+        a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    __shared__ float warp_max[kQuantThreads / 32];
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = a;
+    __syncthreads();
+    a = warp_max[0];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, warp_max[w]);
+
+    const float s = __fdiv_rn(a, 127.0f);
+    if (threadIdx.x == 0) scale[m] = (a == 0.0f) ? 0.0f : s;
+    for (int64_t i = threadIdx.x; i < K4; i += kQuantThreads) {
+        char4 o = make_char4(0, 0, 0, 0);
+        if (a != 0.0f) {
+            const float4 v = xr[i];
+            auto qz = [s](float f) -> signed char {
+                int r = __float2int_rn(__fdiv_rn(f, s));
+                r = r > 127 ? 127 : (r < -127 ? -127 : r);
+                return (signed char)r;
+            };
+            o = make_char4(qz(v.x), qz(v.y), qz(v.z), qz(v.w));
+        }
+        qr[i] = o;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Repack: canonical stream -> kernel-native layout (one thread per word).
+// ---------------------------------------------------------------------------
+__global__ void repack_kernel(const uint8_t* __restrict__ codes, int64_t N, int64_t K, uint32_t* __restrict__ out,
+                              int64_t total_words)
+{
+    const int64_t row_bytes = K / 32 * 5;
+    const int64_t Kc = sherry_k_chunks(K);
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total_words;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = idx % SHERRY_TILE_ROWS;
+        const int64_t j = (idx / SHERRY_TILE_ROWS) % SHERRY_CHUNK_WORDS;
+        const int64_t c = (idx / (SHERRY_TILE_ROWS * SHERRY_CHUNK_WORDS)) % Kc;
+        const int64_t t = idx / (SHERRY_TILE_ROWS * SHERRY_CHUNK_WORDS * Kc);
+        const int64_t n = t * SHERRY_TILE_ROWS + r;
+        const int64_t b0 = c * (SHERRY_CHUNK_WORDS * 4) + 4 * j;
+        uint32_t w = 0;
+        if (n < N) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (b0 + b < row_bytes) w |= (uint32_t)codes[n * row_bytes + b0 + b] << (8 * b);
+        }
+        out[idx] = w;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// SIMT comparison kernel: thread = weight row, MT tokens per CTA, decode
+// through a 32-entry shared table, dp4a against the activations.
+// ---------------------------------------------------------------------------
+constexpr int kSimtMT = 8;
+
+__global__ void __launch_bounds__(SHERRY_TILE_ROWS)
+    simt_gemm_kernel(const int8_t* __restrict__ xq, const float* __restrict__ xs,
+                     const uint32_t* __restrict__ wn, const float* __restrict__ alpha, float* __restrict__ y,
+                     int32_t* __restrict__ acc_out, int64_t M, int64_t N, int64_t K)
+{
+    __shared__ uint32_t table[32];
+    if (threadIdx.x < 32) {
+        const uint32_t c = threadIdx.x, z = c & 3u;
+        uint32_t word = 0, slot = 2;
+        for (uint32_t i = 0; i < 4; ++i) {
+            if (i == z) continue;
+            word |= (((c >> slot) & 1u) ? 0xFFu : 0x01u) << (8 * i);
+            ++slot;
+        }
+        table[c] = word;
+    }
+    __syncthreads();
+    const int64_t t = blockIdx.x;
+    const int r = threadIdx.x;
+    const int64_t n = t * SHERRY_TILE_ROWS + r;
+    const int64_t m0 = (int64_t)blockIdx.y * kSimtMT;
+    const int64_t Kc = sherry_k_chunks(K);
+    int32_t acc[kSimtMT];
+#pragma unroll
+    for (int i = 0; i < kSimtMT; ++i) acc[i] = 0;
+    for (int64_t c = 0; c < Kc; ++c) {
+        const uint32_t* blk = wn + (t * Kc + c) * (SHERRY_TILE_ROWS * SHERRY_CHUNK_WORDS);
+        uint32_t w[SHERRY_CHUNK_WORDS + 1];
+#pragma unroll
+        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) w[j] = blk[j * SHERRY_TILE_ROWS + r];
+        w[SHERRY_CHUNK_WORDS] = 0;
+        for (int g = 0; g < 32; ++g) {
+            const int64_t k = c * SHERRY_KCHUNK + 4 * g;
+            if (k >= K) break;
+            const int bit = 5 * g;
+            const uint32_t v = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31);
+            const int W4 = (int)table[v & 31u];
+#pragma unroll
+            for (int i = 0; i < kSimtMT; ++i) {
+                const int64_t m = m0 + i;
+                if (m < M) acc[i] = __dp4a(W4, *reinterpret_cast<const int*>(xq + m * K + k), acc[i]);
+            }
+        }
+    }
+    if (n >= N) return;
+    const float al = alpha[n];
+#pragma unroll
+    for (int i = 0; i < kSimtMT; ++i) {
+        const int64_t m = m0 + i;
+        if (m >= M) break;
+        if (acc_out) acc_out[m * N + n] = acc[i];
+        if (y) y[m * N + n] = __fmul_rn(__fmul_rn((float)acc[i], al), xs[m]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host helpers
+// ---------------------------------------------------------------------------
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SHERRY_OK : SHERRY_ERR_CUDA; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+struct DeviceInfo {
+    bool checked = false;
+    bool ok = false;
+    int sms = 0;
+    int max_smem_optin = 0;
+};
+
+std::mutex g_mutex;
+std::vector<DeviceInfo> g_dev;
+
+struct Workspace {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+std::vector<Workspace> g_ws;
+
+int device_info(DeviceInfo* out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SHERRY_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.checked) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SHERRY_ERR_CUDA;
+        d.ok = (prop.major == 10 && prop.minor == 0);
+        d.sms = prop.multiProcessorCount;
+        d.max_smem_optin = (int)prop.sharedMemPerBlockOptin;
+        d.checked = true;
+    }
+    *out = d;
+    return d.ok ? SHERRY_OK : SHERRY_ERR_DEVICE;
+}
+
+// Zero-initialised per-device workspace of at least `bytes`, ordered on `stream`.
+int get_workspace(size_t bytes, cudaStream_t stream, void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SHERRY_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((int)g_ws.size() <= dev) g_ws.resize(dev + 1);
+    Workspace& w = g_ws[dev];
+    if (w.bytes < bytes) {
+        if (w.ptr) {
+            if (cudaStreamSynchronize(stream) != cudaSuccess) return SHERRY_ERR_CUDA;
+            cudaFree(w.ptr);
+            w.ptr = nullptr;
+            w.bytes = 0;
+        }
+        size_t nb = std::max<size_t>(bytes, size_t(1) << 20);
+        if (cudaMalloc(&w.ptr, nb) != cudaSuccess) {
+            w.ptr = nullptr;
+            return SHERRY_ERR_CUDA;
+        }
+        if (cudaMemsetAsync(w.ptr, 0, nb, stream) != cudaSuccess) return SHERRY_ERR_CUDA;
+        w.bytes = nb;
+    }
+    *out = w.ptr;
+    return SHERRY_OK;
+}
+
+int make_x_map(CUtensorMap* map, const int8_t* x, int64_t M, int64_t K, int bn)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return SHERRY_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {SHERRY_KCHUNK, (cuuint32_t)bn};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(x), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? SHERRY_OK : SHERRY_ERR_CUDA;
+}
+
+unsigned* device_status_ptr()
+{
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    return static_cast<unsigned*>(p);
+}
+
+template <int BN>
+int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y, int32_t* acc,
+              int64_t M, int64_t N, int64_t K, cudaStream_t stream)
+{
+    using C = tc::Cfg<BN>;
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != SHERRY_OK) return st;
+    tc::Params p;
+    p.wnative = static_cast<const uint8_t*>(wn);
+    p.alpha = alpha;
+    p.x_scale = xs;
+    p.y = y;
+    p.acc = acc;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.TM = (M + BN - 1) / BN;
+    p.TN = sherry_row_tiles(N);
+    p.Kc = sherry_k_chunks(K);
+    p.U = p.TM * p.TN * p.Kc;
+    const int64_t grid = std::min<int64_t>(di.sms, p.U);
+    void* ws = nullptr;
+    const size_t ws_acc = (size_t)grid * BN * SHERRY_TILE_ROWS * sizeof(int32_t);
+    st = get_workspace(ws_acc + (size_t)grid * sizeof(uint32_t), stream, &ws);
+    if (st != SHERRY_OK) return st;
+    p.ws = static_cast<int32_t*>(ws);
+    p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ws_acc);
+    p.status = device_status_ptr();
+    if (!p.status) return SHERRY_ERR_CUDA;
+
+    CUtensorMap map;
+    st = make_x_map(&map, x, M, K, BN);
+    if (st != SHERRY_OK) return st;
+
+    // at least half of the SM's shared memory so that exactly one CTA (and
+    // one 512-column tensor-memory allocation) lives on each SM
+    const int smem = std::max(C::kSmemBytes, 120 * 1024);
+    if (smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
+    cudaError_t e = cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return SHERRY_ERR_CUDA;
+    tc::sherry_gemm_tc_kernel<BN><<<(unsigned)grid, tc::kThreads, smem, stream>>>(map, p);
+    return cuda_status(cudaGetLastError());
+}
+
+int check_gemm_args(const int8_t* x, const float* xs, const void* wn, const float* alpha, const float* y,
+                    const int32_t* acc, int64_t M, int64_t N, int64_t K)
+{
+    if (!x || !xs || !wn || !alpha || (!y && !acc)) return SHERRY_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return SHERRY_ERR_INVALID_ARG;
+    if (!sherry_shape_ok(M, N, K)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(wn)) return SHERRY_ERR_INVALID_ARG;
+    return SHERRY_OK;
+}
+
+}  // namespace
+
+}  // namespace sherry
+
+using namespace sherry;
+
+extern "C" {
+
+int sherry_repack(const uint8_t* codes_dev, int64_t N, int64_t K, void* native_dev, void* stream)
+{
+    if (!codes_dev || !native_dev) return SHERRY_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0) return SHERRY_ERR_INVALID_ARG;
+    if (!sherry_shape_ok(1, N, K)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(native_dev)) return SHERRY_ERR_INVALID_ARG;
+    const int64_t words = (int64_t)(sherry_native_bytes(N, K) / 4);
+    const int threads = 256;
+    const int64_t blocks = std::min<int64_t>((words + threads - 1) / threads, 148 * 32);
+    repack_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        codes_dev, N, K, static_cast<uint32_t*>(native_dev), words);
+    return cuda_status(cudaGetLastError());
+}
+
+int sherry_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_i8, float* x_scale, void* stream)
+{
+    if (!x || !x_i8 || !x_scale) return SHERRY_ERR_INVALID_ARG;
+    if (M <= 0 || K <= 0) return SHERRY_ERR_INVALID_ARG;
+    if (!sherry_shape_ok(M, 1, K)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(x_i8)) return SHERRY_ERR_INVALID_ARG;
+    quant_act_kernel<<<(unsigned)M, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(x, K, x_i8, x_scale);
+    return cuda_status(cudaGetLastError());
+}
+
+int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,
+                    int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
+    if (st != SHERRY_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= 16) return launch_tc<16>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    if (M <= 32) return launch_tc<32>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    if (M <= 64) return launch_tc<64>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    return launch_tc<128>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+}
+
+int sherry_gemm(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,
+                int64_t M, int64_t N, int64_t K, void* stream)
+{
+    if (!y) return SHERRY_ERR_INVALID_ARG;
+    return sherry_gemm_acc(x_i8, x_scale, Wnative, alpha, y, nullptr, M, N, K, stream);
+}
+
+int sherry_gemm_simt(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,
+                     int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
+    if (st != SHERRY_OK) return st;
+    DeviceInfo di;
+    st = device_info(&di);
+    if (st != SHERRY_OK) return st;
+    dim3 grid((unsigned)sherry_row_tiles(N), (unsigned)((M + kSimtMT - 1) / kSimtMT));
+    if ((M + kSimtMT - 1) / kSimtMT > 65535) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    simt_gemm_kernel<<<grid, SHERRY_TILE_ROWS, 0, static_cast<cudaStream_t>(stream)>>>(
+        x_i8, x_scale, static_cast<const uint32_t*>(Wnative), alpha, y, acc, M, N, K);
+    return cuda_status(cudaGetLastError());
+}
+
+int sherry_last_device_status(int reset)
+{
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return -1;
+    if (reset) {
+        unsigned z = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(z)) != cudaSuccess) return -1;
+    }
+    return (int)v;
+}
+
+}  // extern "C"

@@ -1,0 +1,412 @@
+// Sherry 3:4 ternary GEMM on the sm_100a tensor cores.
+//
+// What it computes (Sherry page, pnsm.cn/news/1195499, sec. 2.2 steps 2-4):
+//   acc[m][n] = sum_k x_i8[m][k] * T[n][k]           (exact int32)
+//   y[m][n]   = (float)((float)acc[m][n] * alpha[n]) * x_scale[m]
+// with T decoded from the 5-bit group codes of sec. 2.1.
+//
+// How (the page's CPU/Jetson table-lookup kernels are prior art only): the
+// problem is run "swap-AB" on tcgen05.mma.kind::i8 with M = 128 weight rows,
+// N = BN tokens and K = 32 per instruction.
+//   * A (weights) lives in tensor memory.  Decoder warps read the packed
+//     codes of their row from shared memory, turn every 5-bit code into the
+//     four int8 weights {-1,0,+1} of its group with one lookup in a 32-entry
+//     table, and store them with tcgen05.st: one 32-bit TMEM cell is one
+//     group, so a 128-wide K chunk of a row is 32 consecutive columns of that
+//     row's lane.
+//   * B (activations) is loaded by TMA into shared memory, K-major with the
+//     128-byte swizzle, and described to the MMA by a shared-memory matrix
+//     descriptor; rows past M and columns past K are zero-filled by TMA.
+//   * D (int32 accumulators) lives in tensor memory; epilogue warps read it
+//     with tcgen05.ld and apply the two fp32 products.
+// Work is split "stream-K": the (token tile, row tile, K chunk) units are
+// cut into one contiguous range per CTA (one CTA per SM), so every SM gets
+// the same number of K chunks whatever the shape.  A tile whose K range spans
+// several CTAs is summed exactly with int32 red.add into a workspace slot;
+// the last contributor (an atomic counter) runs the epilogue and clears the
+// slot and counter, so the workspace is all zero between calls.
+//
+// Warp roles (512 threads):
+//   warp 0       producer: one bulk copy of 128 rows x 20 bytes of codes and
+//                one 2D TMA of the activation tile per K chunk
+//   warp 1       TMEM allocation and MMA issue (one thread)
+//   warps 4-11   two decoder groups of four warps (one warp per TMEM lane
+//                quadrant), alternating K chunks
+//   warps 12-15  epilogue (one warp per lane quadrant)
+// Every wait is bounded in wall time; when a bound runs out the kernel
+// records a status code, stops issuing work, waits (bounded) for what it has
+// in flight, frees its tensor memory and returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "ptx.cuh"
+#include "sherry_internal.h"
+
+namespace sherry {
+namespace tc {
+
+constexpr int kThreads = 512;
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kDecWarp0 = 4;
+constexpr int kDecGroups = 2;
+constexpr int kEpiWarp0 = 12;
+constexpr int kTmemCols = 512;
+constexpr int kCodeStageBytes = SHERRY_CHUNK_BYTES_PER_TILE;   // 2560
+constexpr uint64_t kWaitLimitNs = 2000000000ull;              // 2 s per wait
+
+template <int BN>
+struct Cfg {
+    static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
+    static constexpr int kBStageBytes = BN * 128;
+    static constexpr int kStageBytes = kBStageBytes + kCodeStageBytes;
+    static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 24 ? 24 : kStagesRaw;
+    static constexpr int kDBufs = (2 * BN + 8 * 32 <= kTmemCols) ? 2 : 1;
+    static constexpr int kAStagesRaw = (kTmemCols - kDBufs * BN) / 32;
+    static constexpr int kAStages = kAStagesRaw > 12 ? 12 : kAStagesRaw;
+    static constexpr int kACol0 = kDBufs * BN;
+    // shared memory: [B stages][code stages][barriers + misc]
+    static constexpr int kOffCodes = kStages * kBStageBytes;
+    static constexpr int kOffBars = kOffCodes + kStages * kCodeStageBytes;
+    static constexpr int kNumBars = 2 * kStages + 2 * kAStages + 2 * kDBufs + 1;
+    static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
+    static constexpr int kMiscBytes = 64 + 32 * 4;   // tmem holder, flags, decode table
+    static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;   // + alignment slack
+    // instruction descriptor: s32 accumulate, signed int8 A and B, both
+    // K-major, N = BN, M = 128
+    static constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
+                                       (uint32_t(128 >> 4) << 24);
+};
+
+struct Params {
+    const uint8_t* wnative;     // kernel-native codes
+    const float* alpha;         // [N]
+    const float* x_scale;       // [M]
+    float* y;                   // [M][N] or null
+    int32_t* acc;               // [M][N] or null
+    int32_t* ws;                // split-K slots [grid][BN][128]
+    uint32_t* counters;         // [grid]
+    unsigned* status;           // device status word
+    int64_t M, N, K;
+    int64_t TM, TN, Kc;         // token tiles, row tiles, K chunks
+    int64_t U;                  // total units TM*TN*Kc
+};
+
+// CTA that owns unit u when U units are cut into G contiguous ranges
+// [floor(U b / G), floor(U (b+1) / G)).
+__device__ __forceinline__ int64_t owner_of(int64_t u, int64_t U, int64_t G)
+{
+    return ((u + 1) * G - 1) / U;
+}
+
+__device__ __forceinline__ uint64_t b_desc_sw128(uint32_t smem_addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);          // start address
+    d |= (uint64_t)1u << 16;                               // leading byte offset (unused, 16 B)
+    d |= (uint64_t)(1024u >> 4) << 32;                     // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1u << 46;                               // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                               // 128-byte swizzle
+    return d;
+}
+
+__device__ __forceinline__ void report(unsigned* status, volatile int* abort_flag, unsigned code)
+{
+    atomicCAS(status, 0u, code);
+    *abort_flag = 1;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    sherry_gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p)
+{
+    using C = Cfg<BN>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const uint32_t bar0 = sbase + C::kOffBars;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+    auto afull_bar = [&](int a) { return bar0 + 8u * (2 * C::kStages + a); };
+    auto aempty_bar = [&](int a) { return bar0 + 8u * (2 * C::kStages + C::kAStages + a); };
+    auto dfull_bar = [&](int d) { return bar0 + 8u * (2 * C::kStages + 2 * C::kAStages + d); };
+    auto dempty_bar = [&](int d) { return bar0 + 8u * (2 * C::kStages + 2 * C::kAStages + C::kDBufs + d); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 2 * C::kAStages + 2 * C::kDBufs);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
+    volatile int* go_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);   // [2]
+    uint32_t* table = reinterpret_cast<uint32_t*>(smem + C::kOffMisc + 64);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // this CTA's unit range
+    const int64_t G = gridDim.x;
+    const int64_t u0 = (p.U * (int64_t)blockIdx.x) / G;
+    const int64_t u1 = (p.U * ((int64_t)blockIdx.x + 1)) / G;
+    const int64_t n_it = u1 - u0;
+
+    if (threadIdx.x < 32) {
+        // code -> four int8 weights of the group, byte i = position i
+        const uint32_t c = threadIdx.x, z = c & 3u;
+        uint32_t word = 0, slot = 2;
+        for (uint32_t i = 0; i < 4; ++i) {
+            uint32_t b = 0;
+            if (i != z) {
+                b = ((c >> slot) & 1u) ? 0xFFu : 0x01u;
+                ++slot;
+            }
+            word |= b << (8 * i);
+        }
+        table[c] = word;
+    }
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < C::kStages; ++s) {
+            ptx::mbar_init(full_bar(s), 1);
+            ptx::mbar_init(empty_bar(s), 4 + 1);
+        }
+        for (int a = 0; a < C::kAStages; ++a) {
+            ptx::mbar_init(afull_bar(a), 4);
+            ptx::mbar_init(aempty_bar(a), 1);
+        }
+        for (int d = 0; d < C::kDBufs; ++d) {
+            ptx::mbar_init(dfull_bar(d), 1);
+            ptx::mbar_init(dempty_bar(d), 4);
+        }
+        ptx::mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_holder), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (threadIdx.x == 0) ptx::prefetch_tensormap(&xmap);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            int64_t issued = 0;
+            for (int64_t it = 0; it < n_it && !*abort_flag; ++it) {
+                const int s = (int)(it % C::kStages);
+                const uint32_t ph = (uint32_t)((it / C::kStages) & 1);
+                if (!ptx::mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs)) {
+                    report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_PRODUCER);
+                    break;
+                }
+                const int64_t u = u0 + it;
+                const int64_t tile = u / p.Kc, c = u % p.Kc;
+                const int64_t tm = tile / p.TN, tn = tile % p.TN;
+                ptx::mbar_arrive_expect_tx(full_bar(s), (uint32_t)(kCodeStageBytes + C::kBStageBytes));
+                ptx::bulk_g2s(sbase + C::kOffCodes + (uint32_t)s * kCodeStageBytes,
+                              p.wnative + (tn * p.Kc + c) * (int64_t)kCodeStageBytes, kCodeStageBytes,
+                              full_bar(s));
+                ptx::tma_load_2d(sbase + (uint32_t)s * C::kBStageBytes, &xmap, (int32_t)(c * SHERRY_KCHUNK),
+                                 (int32_t)(tm * BN), full_bar(s));
+                ++issued;
+            }
+            // every copy issued has landed before the CTA may exit (in the
+            // normal flow the consumers already waited for all of them)
+            const int64_t from = issued > C::kStages ? issued - C::kStages : 0;
+            for (int64_t i = from; i < issued; ++i)
+                if (!ptx::mbar_wait_bounded(full_bar((int)(i % C::kStages)), (uint32_t)((i / C::kStages) & 1),
+                                            kWaitLimitNs)) {
+                    atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
+                    break;
+                }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            int64_t it = 0, seg = 0;
+            bool issued_any = false;
+            int64_t u = u0;
+            while (u < u1 && !*abort_flag) {
+                const int64_t tile = u / p.Kc;
+                const int64_t seg_end = (tile + 1) * p.Kc < u1 ? (tile + 1) * p.Kc : u1;
+                const int d = (int)(seg % C::kDBufs);
+                if (!ptx::mbar_wait_bounded(dempty_bar(d), (uint32_t)(((seg / C::kDBufs) & 1) ^ 1),
+                                            kWaitLimitNs)) {
+                    report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
+                bool first = true;
+                for (; u < seg_end; ++u, ++it) {
+                    const int s = (int)(it % C::kStages);
+                    const int a = (int)(it % C::kAStages);
+                    if (!ptx::mbar_wait_bounded(full_bar(s), (uint32_t)((it / C::kStages) & 1), kWaitLimitNs) ||
+                        !ptx::mbar_wait_bounded(afull_bar(a), (uint32_t)((it / C::kAStages) & 1), kWaitLimitNs)) {
+                        report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a_tmem = tmem + (uint32_t)(C::kACol0 + a * 32);
+                    const uint32_t b_addr = sbase + (uint32_t)s * C::kBStageBytes;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        ptx::mma_i8_ts(d_tmem, a_tmem + 8u * ks, b_desc_sw128(b_addr + 32u * ks), C::kIdesc,
+                                       (first && ks == 0) ? 0u : 1u);
+                    }
+                    issued_any = true;
+                    first = false;
+                    ptx::tc_commit(empty_bar(s));
+                    ptx::tc_commit(aempty_bar(a));
+                }
+                if (*abort_flag) break;
+                ptx::tc_commit(dfull_bar(d));
+                ++seg;
+            }
+            if (issued_any) {
+                // all MMAs of this thread complete before tensor memory is freed
+                ptx::tc_commit(drain_bar);
+                if (!ptx::mbar_wait_bounded(drain_bar, 0, kWaitLimitNs))
+                    atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
+            }
+        }
+    } else if (warp >= kDecWarp0 && warp < kDecWarp0 + 4 * kDecGroups) {
+        const int grp = (warp - kDecWarp0) / 4;
+        const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+        const int row = quad * 32 + lane;          // row within the 128-row tile
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        for (int64_t it = grp; it < n_it; it += kDecGroups) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            const int s = (int)(it % C::kStages);
+            bool ok = ptx::mbar_wait_bounded(full_bar(s), (uint32_t)((it / C::kStages) & 1), kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
+                break;
+            }
+            const uint32_t* codes =
+                reinterpret_cast<const uint32_t*>(smem + C::kOffCodes + s * kCodeStageBytes);
+            uint32_t w[SHERRY_CHUNK_WORDS];
+#pragma unroll
+            for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) w[j] = codes[j * SHERRY_TILE_ROWS + row];
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(empty_bar(s));
+            uint32_t a_vals[32];
+#pragma unroll
+            for (int g = 0; g < 32; ++g) {
+                const int bit = 5 * g, wi = bit >> 5, off = bit & 31;
+                uint32_t v;
+                if (off <= 27) v = w[wi] >> off;
+                else v = __funnelshift_r(w[wi], w[wi + 1], off);
+                a_vals[g] = table[v & 31u];
+            }
+            const int a = (int)(it % C::kAStages);
+            ok = ptx::mbar_wait_bounded(aempty_bar(a), (uint32_t)(((it / C::kAStages) & 1) ^ 1), kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
+                break;
+            }
+            ptx::tc_fence_after();
+            ptx::tmem_st_32x32b_x32(lane_base + (uint32_t)(C::kACol0 + a * 32), a_vals);
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(afull_bar(a));
+        }
+    } else if (warp >= kEpiWarp0) {
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        const int etid = threadIdx.x - kEpiWarp0 * 32;     // 0..127
+        int64_t seg = 0;
+        int64_t u = u0;
+        while (u < u1) {
+            const int64_t tile = u / p.Kc;
+            const int64_t cb = u - tile * p.Kc;
+            const int64_t seg_end = (tile + 1) * p.Kc < u1 ? (tile + 1) * p.Kc : u1;
+            const int64_t ce = seg_end - tile * p.Kc;
+            u = seg_end;
+            const int64_t tm = tile / p.TN, tn = tile % p.TN;
+            const int64_t n = tn * SHERRY_TILE_ROWS + r;
+            const bool complete = (cb == 0 && ce == p.Kc);
+            const int d = (int)(seg % C::kDBufs);
+            // one thread waits, the decision is shared through a named barrier
+            // so that all 128 epilogue threads leave or stay together
+            if (etid == 0) {
+                bool ok = !*abort_flag &&
+                          ptx::mbar_wait_bounded(dfull_bar(d), (uint32_t)((seg / C::kDBufs) & 1), kWaitLimitNs);
+                if (!ok && !*abort_flag) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_EPILOGUE);
+                go_flag[seg & 1] = ok ? 1 : 0;
+            }
+            ptx::named_bar_sync(1, 128);
+            if (!go_flag[seg & 1]) break;
+            ptx::tc_fence_after();
+            const float al = (n < p.N) ? p.alpha[n] : 0.0f;
+            int64_t slot = 0, nparts = 1;
+            if (!complete) {
+                const int64_t bf = owner_of(tile * p.Kc, p.U, G);
+                const int64_t bl = owner_of(tile * p.Kc + p.Kc - 1, p.U, G);
+                slot = bf;
+                nparts = bl - bf + 1;
+            }
+            int32_t* wsl = p.ws + slot * (int64_t)BN * SHERRY_TILE_ROWS;
+#pragma unroll 1
+            for (int j0 = 0; j0 < BN; j0 += 16) {
+                uint32_t v[16];
+                ptx::tmem_ld_32x32b_x16(lane_base + (uint32_t)(d * BN + j0), v);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int64_t m = tm * BN + j0 + jj;
+                    if (m >= p.M) continue;
+                    const int32_t a32 = (int32_t)v[jj];
+                    if (complete) {
+                        if (n < p.N) {
+                            if (p.acc) p.acc[m * p.N + n] = a32;
+                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, al), p.x_scale[m]);
+                        }
+                    } else {
+                        ptx::red_add_s32(wsl + (j0 + jj) * SHERRY_TILE_ROWS + r, a32);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(dempty_bar(d));
+            ++seg;
+            if (!complete) {
+                __threadfence();
+                ptx::named_bar_sync(1, 128);
+                if (etid == 0) {
+                    const uint32_t old = atomicAdd(p.counters + slot, 1u);
+                    *last_flag = (old == (uint32_t)(nparts - 1)) ? 1 : 0;
+                }
+                ptx::named_bar_sync(1, 128);
+                if (*last_flag) {
+                    __threadfence();
+                    for (int j = 0; j < BN; ++j) {
+                        const int64_t m = tm * BN + j;
+                        if (m >= p.M) break;
+                        int32_t* cell = wsl + j * SHERRY_TILE_ROWS + r;
+                        const int32_t a32 = ptx::ld_cg_s32(cell);
+                        *cell = 0;
+                        if (n < p.N) {
+                            if (p.acc) p.acc[m * p.N + n] = a32;
+                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, al), p.x_scale[m]);
+                        }
+                    }
+                    if (etid == 0) atomicExch(p.counters + slot, 0u);
+                }
+                ptx::named_bar_sync(1, 128);
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace tc
+}  // namespace sherry

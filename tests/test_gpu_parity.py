@@ -1,0 +1,158 @@
+"""GPU parity: every step of the CUDA path against the oracle, through the C ABI.
+
+Bar: int8 activations, scales and int32 accumulators bit-exact; fp32 outputs
+within 1e-6 relative (they are expected bit-identical).  Small ragged shapes
+are compared in full; the five workload configurations run at full size with
+oracle rows sampled at tile edges and at random, plus a full comparison of
+the accumulators with torch._int_mm (a library int8 GEMM) over the oracle's
+ternary weights where its shape rules allow (M > 16)."""
+import numpy as np
+import pytest
+
+import oracle
+import sparse_bit_matmul_b200 as sbm
+import synth
+from sherry_testlib import assert_y_close, rows_sample, run_gpu, upload_weights
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    sbm.load()
+    assert sbm.last_device_status(reset=True) >= 0
+    yield
+    assert sbm.last_device_status() == 0
+
+
+# ------------------------------------------------------------ quantiser
+@pytest.mark.parametrize("M,K,cfg", [(1, 256, 0), (3, 4096, 1), (32, 14336, 2), (128, 8192, 4), (5, 32, 0)])
+def test_quant_act_bitexact(M, K, cfg):
+    x = synth.config_activations(cfg, 0, M, K)
+    q_o, s_o = oracle.quant_act(x)
+    q, s = sbm.quant_act(torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_o)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+
+
+def test_quant_act_ties_and_zero_rows():
+    s = 0.125
+    j = np.arange(-126, 126)
+    row = np.concatenate([[127 * s], (j + 0.5) * s, np.zeros(32 - (1 + len(j)) % 32)]).astype(np.float32)
+    x = np.stack([row, np.zeros_like(row), -row]).astype(np.float32)
+    q_o, s_o = oracle.quant_act(x)
+    q, sc = sbm.quant_act(torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_o)
+    assert np.array_equal(sc.cpu().numpy(), s_o)
+
+
+# --------------------------------------------------------------- repack
+@pytest.mark.parametrize("N,K", [(300, 96), (128, 4096), (129, 224), (1, 32)])
+def test_repack_layout(N, K):
+    rng = np.random.default_rng(N + K)
+    codes = rng.integers(0, 256, size=(N, K // 32 * 5), dtype=np.uint8)
+    nat = sbm.repack(torch.from_numpy(codes).cuda(), N, K).cpu().numpy().view(np.uint32)
+    Tn, Kc = -(-N // 128), -(-K // 128)
+    assert nat.size == Tn * Kc * 5 * 128
+    pad = np.zeros((Tn * 128, Kc * 20), dtype=np.uint8)
+    pad[:N, :codes.shape[1]] = codes
+    expect = pad.reshape(Tn, 128, Kc, 5, 4).view(np.uint32)[..., 0]      # [t][r][c][j]
+    expect = expect.transpose(0, 2, 3, 1).reshape(-1)                   # [t][c][j][r]
+    assert np.array_equal(nat, expect)
+
+
+# ---------------------------------------------- small ragged shapes, full
+SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 512),
+         (64, 256, 1024), (100, 130, 4096), (129, 257, 160), (256, 512, 2048), (7, 1, 32)]
+
+
+@pytest.mark.parametrize("kernel", ["tc", "simt"])
+@pytest.mark.parametrize("M,N,K", SMALL)
+def test_gemm_small_full(M, N, K, kernel):
+    W = synth.weights(0, 1, N, K, sigma=0.02)
+    x = synth.activations(0, 1, M, K)
+    y_o, acc_o, q_o, s_o, codes_o, alpha_o = oracle.reference(x, W)
+    native, alpha_d, codes, alpha = upload_weights(W)
+    assert np.array_equal(codes, codes_o) and np.array_equal(alpha, alpha_o)
+    y, acc, q, s = run_gpu(x, native, alpha_d, N, kernel)
+    assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
+    assert np.array_equal(acc, acc_o)
+    assert_y_close(y, y_o)
+
+
+def test_gemm_zero_token_and_repeat():
+    """all-zero token -> y = 0; repeated calls agree (workspace left clean)."""
+    N, K = 300, 1024
+    W = synth.weights(0, 2, N, K)
+    x = synth.activations(0, 2, 5, K)
+    x[2] = 0.0
+    native, alpha_d, _, _ = upload_weights(W)
+    first = run_gpu(x, native, alpha_d, N)
+    assert np.all(first[0][2] == 0) and np.all(first[1][2] == 0)
+    for _ in range(3):
+        again = run_gpu(x, native, alpha_d, N)
+        assert np.array_equal(again[1], first[1]) and np.array_equal(again[0], first[0])
+    y_o, acc_o, *_ = oracle.reference(x, W)
+    assert np.array_equal(first[1], acc_o)
+
+
+# ----------------------------------------------- full-size configurations
+def _full_size_check(cfg, copy, M_list, K, N, int_mm=True):
+    W = synth.config_weights(cfg, copy, K, N)
+    native, alpha_d, codes, alpha = upload_weights(W)
+    rows = rows_sample(N, seed=cfg * 7 + N)
+    T_rows, a_rows = oracle.quantise(W[rows])
+    assert np.array_equal(codes[rows], oracle.pack(T_rows))
+    assert np.array_equal(alpha[rows], a_rows)
+    T_full = None
+    for M in M_list:
+        x = synth.config_activations(cfg, copy, M, K)
+        q_o, s_o = oracle.quant_act(x)
+        y, acc, q, s = run_gpu(x, native, alpha_d, N)
+        assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
+        acc_o = oracle.gemm(q_o, T_rows)
+        assert np.array_equal(acc[:, rows], acc_o)
+        assert_y_close(y[:, rows], oracle.epilogue(acc_o, a_rows, s_o))
+        if int_mm and M > 16:
+            if T_full is None:
+                T_full, _ = oracle.quantise(W)
+            ref = torch._int_mm(torch.from_numpy(q_o).cuda(), torch.from_numpy(T_full).cuda().t().contiguous())
+            assert torch.equal(torch.from_numpy(acc).cuda(), ref)
+    return W
+
+
+@pytest.mark.parametrize("K,N", synth.PROJ_SHAPES)
+def test_config1_decode_full_size(K, N):
+    _full_size_check(1, 0, [1], K, N)
+
+
+@pytest.mark.parametrize("K,N", synth.PROJ_SHAPES)
+def test_config2_small_batch_full_size(K, N):
+    _full_size_check(2, 0, [4, 8, 16, 32], K, N)
+
+
+@pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096)])
+def test_config3_prefill_full_size(K, N):
+    _full_size_check(3, 0, [2048], K, N)
+
+
+def test_config4_heavy_tail_full_size():
+    W = _full_size_check(4, 0, [1, 128, 4096], 8192, 28672)
+    T, _ = oracle.quantise(W)
+    assert np.all(np.count_nonzero(T.reshape(28672, -1, 4), axis=2) == 3)
+
+
+def test_config0_tiny_exact():
+    W = synth.config_weights(0, 0, 256, 128)
+    x = synth.config_activations(0, 0, 1, 256)
+    y_o, acc_o, *_ = oracle.reference(x, W)
+    native, alpha_d, _, _ = upload_weights(W)
+    for kernel in ("tc", "simt"):
+        y, acc, _, _ = run_gpu(x, native, alpha_d, 128, kernel)
+        assert np.array_equal(acc, acc_o)
+        assert np.array_equal(y, y_o)
