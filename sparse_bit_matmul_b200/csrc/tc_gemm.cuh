@@ -26,13 +26,15 @@
 // the last contributor (an atomic counter) runs the epilogue and clears the
 // slot and counter, so the workspace is all zero between calls.
 //
-// Warp roles (512 threads):
+// Warp roles (576 threads):
 //   warp 0       producer: one bulk copy of 128 rows x 20 bytes of codes and
 //                one 2D TMA of the activation tile per K chunk
 //   warp 1       TMEM allocation and MMA issue (one thread)
-//   warps 4-11   two decoder groups of four warps (one warp per TMEM lane
-//                quadrant), alternating K chunks
-//   warps 12-15  epilogue (one warp per lane quadrant)
+//   warps 2-13   three decoder groups of four warps (each group covers the
+//                four TMEM lane quadrants), taking K chunks in turn
+//   warps 14-17  epilogue (one warp per lane quadrant)
+// Loop indices (stage, phase, tile coordinates) advance incrementally: no
+// integer division on the per-chunk path.
 // Every wait is bounded in wall time; when a bound runs out the kernel
 // records a status code, stops issuing work, waits (bounded) for what it has
 // in flight, frees its tensor memory and returns.
@@ -47,12 +49,12 @@
 namespace sherry {
 namespace tc {
 
-constexpr int kThreads = 512;
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
-constexpr int kDecWarp0 = 4;
-constexpr int kDecGroups = 2;
-constexpr int kEpiWarp0 = 12;
+constexpr int kDecWarp0 = 2;
+constexpr int kDecGroups = 3;
+constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;
+constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kTmemCols = 512;
 constexpr int kCodeStageBytes = SHERRY_CHUNK_BYTES_PER_TILE;   // 2560
 constexpr uint64_t kWaitLimitNs = 2000000000ull;              // 2 s per wait
@@ -73,7 +75,7 @@ struct Cfg {
     static constexpr int kOffBars = kOffCodes + kStages * kCodeStageBytes;
     static constexpr int kNumBars = 2 * kStages + 2 * kAStages + 2 * kDBufs + 1;
     static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
-    static constexpr int kMiscBytes = 64 + 32 * 4;   // tmem holder, flags, decode table
+    static constexpr int kMiscBytes = 64;            // tmem holder, flags
     static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;   // + alignment slack
     // instruction descriptor: s32 accumulate, signed int8 A and B, both
     // K-major, N = BN, M = 128
@@ -125,7 +127,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     using C = Cfg<BN>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(128) uint32_t table[32];
+    // 1024-byte aligned start, computed by pointer arithmetic so that the
+    // compiler keeps the shared address space (plain ld.shared/st.shared)
+    uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar0 = sbase + C::kOffBars;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -139,7 +144,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
     volatile int* go_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);   // [2]
-    uint32_t* table = reinterpret_cast<uint32_t*>(smem + C::kOffMisc + 64);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -194,16 +198,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kProducerWarp) {
         if (lane == 0) {
             int64_t issued = 0;
+            int64_t tile = u0 / p.Kc, c = u0 - (u0 / p.Kc) * p.Kc;
+            int64_t tm = tile / p.TN, tn = tile - (tile / p.TN) * p.TN;
+            int s = 0;
+            uint32_t ph = 0;
             for (int64_t it = 0; it < n_it && !*abort_flag; ++it) {
-                const int s = (int)(it % C::kStages);
-                const uint32_t ph = (uint32_t)((it / C::kStages) & 1);
                 if (!ptx::mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs)) {
                     report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_PRODUCER);
                     break;
                 }
-                const int64_t u = u0 + it;
-                const int64_t tile = u / p.Kc, c = u % p.Kc;
-                const int64_t tm = tile / p.TN, tn = tile % p.TN;
                 ptx::mbar_arrive_expect_tx(full_bar(s), (uint32_t)(kCodeStageBytes + C::kBStageBytes));
                 ptx::bulk_g2s(sbase + C::kOffCodes + (uint32_t)s * kCodeStageBytes,
                               p.wnative + (tn * p.Kc + c) * (int64_t)kCodeStageBytes, kCodeStageBytes,
@@ -211,39 +214,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tma_load_2d(sbase + (uint32_t)s * C::kBStageBytes, &xmap, (int32_t)(c * SHERRY_KCHUNK),
                                  (int32_t)(tm * BN), full_bar(s));
                 ++issued;
+                if (++s == C::kStages) { s = 0; ph ^= 1u; }
+                if (++c == p.Kc) {
+                    c = 0;
+                    if (++tn == p.TN) { tn = 0; ++tm; }
+                }
             }
             // every copy issued has landed before the CTA may exit (in the
             // normal flow the consumers already waited for all of them)
             const int64_t from = issued > C::kStages ? issued - C::kStages : 0;
-            for (int64_t i = from; i < issued; ++i)
-                if (!ptx::mbar_wait_bounded(full_bar((int)(i % C::kStages)), (uint32_t)((i / C::kStages) & 1),
-                                            kWaitLimitNs)) {
+            int ds = (int)(from % C::kStages);
+            uint32_t dph = (uint32_t)((from / C::kStages) & 1);
+            for (int64_t i = from; i < issued; ++i) {
+                if (!ptx::mbar_wait_bounded(full_bar(ds), dph, kWaitLimitNs)) {
                     atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
                     break;
                 }
+                if (++ds == C::kStages) { ds = 0; dph ^= 1u; }
+            }
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
-            int64_t it = 0, seg = 0;
+            int64_t seg = 0;
+            int s = 0, a = 0, d = 0;
+            uint32_t sph = 0, aph = 0, dph = 0;
             bool issued_any = false;
             int64_t u = u0;
+            int64_t tile_end = (u0 / p.Kc + 1) * p.Kc;
             while (u < u1 && !*abort_flag) {
-                const int64_t tile = u / p.Kc;
-                const int64_t seg_end = (tile + 1) * p.Kc < u1 ? (tile + 1) * p.Kc : u1;
-                const int d = (int)(seg % C::kDBufs);
-                if (!ptx::mbar_wait_bounded(dempty_bar(d), (uint32_t)(((seg / C::kDBufs) & 1) ^ 1),
-                                            kWaitLimitNs)) {
+                const int64_t seg_end = tile_end < u1 ? tile_end : u1;
+                if (!ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs)) {
                     report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
                     break;
                 }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
                 bool first = true;
-                for (; u < seg_end; ++u, ++it) {
-                    const int s = (int)(it % C::kStages);
-                    const int a = (int)(it % C::kAStages);
-                    if (!ptx::mbar_wait_bounded(full_bar(s), (uint32_t)((it / C::kStages) & 1), kWaitLimitNs) ||
-                        !ptx::mbar_wait_bounded(afull_bar(a), (uint32_t)((it / C::kAStages) & 1), kWaitLimitNs)) {
+                for (; u < seg_end; ++u) {
+                    if (!ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs) ||
+                        !ptx::mbar_wait_bounded(afull_bar(a), aph, kWaitLimitNs)) {
                         report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
                         break;
                     }
@@ -259,9 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     first = false;
                     ptx::tc_commit(empty_bar(s));
                     ptx::tc_commit(aempty_bar(a));
+                    if (++s == C::kStages) { s = 0; sph ^= 1u; }
+                    if (++a == C::kAStages) { a = 0; aph ^= 1u; }
                 }
                 if (*abort_flag) break;
                 ptx::tc_commit(dfull_bar(d));
+                if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
+                tile_end += p.Kc;
                 ++seg;
             }
             if (issued_any) {
@@ -276,10 +289,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;                 // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;          // row within the 128-row tile
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint8_t* tbl = reinterpret_cast<const uint8_t*>(table);
+        // stage and phase of iteration it = grp, grp + G, grp + 2G, ...
+        int s = grp % C::kStages, a = grp % C::kAStages;
+        uint32_t sph = (uint32_t)((grp / C::kStages) & 1), aph = (uint32_t)((grp / C::kAStages) & 1);
         for (int64_t it = grp; it < n_it; it += kDecGroups) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            const int s = (int)(it % C::kStages);
-            bool ok = ptx::mbar_wait_bounded(full_bar(s), (uint32_t)((it / C::kStages) & 1), kWaitLimitNs);
+            bool ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
                 break;
@@ -294,14 +310,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t a_vals[32];
 #pragma unroll
             for (int g = 0; g < 32; ++g) {
+                // byte offset of the group's table entry: code * 4
                 const int bit = 5 * g, wi = bit >> 5, off = bit & 31;
                 uint32_t v;
-                if (off <= 27) v = w[wi] >> off;
-                else v = __funnelshift_r(w[wi], w[wi + 1], off);
-                a_vals[g] = table[v & 31u];
+                if (off == 0) v = w[wi] << 2;
+                else if (off == 1) v = w[wi] << 1;
+                else if (off <= 27) v = w[wi] >> (off - 2);
+                else v = __funnelshift_r(w[wi], w[wi + 1], off - 2);
+                a_vals[g] = *reinterpret_cast<const uint32_t*>(tbl + (v & 0x7Cu));
             }
-            const int a = (int)(it % C::kAStages);
-            ok = ptx::mbar_wait_bounded(aempty_bar(a), (uint32_t)(((it / C::kAStages) & 1) ^ 1), kWaitLimitNs);
+            ok = ptx::mbar_wait_bounded(aempty_bar(a), aph ^ 1u, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
                 break;
@@ -312,6 +330,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(afull_bar(a));
+            s += kDecGroups;
+            if (s >= C::kStages) { s -= C::kStages; sph ^= 1u; }
+            a += kDecGroups;
+            if (a >= C::kAStages) { a -= C::kAStages; aph ^= 1u; }
         }
     } else if (warp >= kEpiWarp0) {
         const int quad = warp & 3;
@@ -320,21 +342,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int etid = threadIdx.x - kEpiWarp0 * 32;     // 0..127
         int64_t seg = 0;
         int64_t u = u0;
+        int64_t tile = u0 / p.Kc;
+        int64_t tm = tile / p.TN, tn = tile - (tile / p.TN) * p.TN;
+        int d = 0;
+        uint32_t dph = 0;
         while (u < u1) {
-            const int64_t tile = u / p.Kc;
             const int64_t cb = u - tile * p.Kc;
             const int64_t seg_end = (tile + 1) * p.Kc < u1 ? (tile + 1) * p.Kc : u1;
             const int64_t ce = seg_end - tile * p.Kc;
             u = seg_end;
-            const int64_t tm = tile / p.TN, tn = tile % p.TN;
             const int64_t n = tn * SHERRY_TILE_ROWS + r;
             const bool complete = (cb == 0 && ce == p.Kc);
-            const int d = (int)(seg % C::kDBufs);
             // one thread waits, the decision is shared through a named barrier
             // so that all 128 epilogue threads leave or stay together
             if (etid == 0) {
-                bool ok = !*abort_flag &&
-                          ptx::mbar_wait_bounded(dfull_bar(d), (uint32_t)((seg / C::kDBufs) & 1), kWaitLimitNs);
+                bool ok = !*abort_flag && ptx::mbar_wait_bounded(dfull_bar(d), dph, kWaitLimitNs);
                 if (!ok && !*abort_flag) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_EPILOGUE);
                 go_flag[seg & 1] = ok ? 1 : 0;
             }
@@ -374,6 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(dempty_bar(d));
             ++seg;
+            if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
+            const int64_t cur_tm = tm;
+            ++tile;
+            if (++tn == p.TN) { tn = 0; ++tm; }
             if (!complete) {
                 __threadfence();
                 ptx::named_bar_sync(1, 128);
@@ -385,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (*last_flag) {
                     __threadfence();
                     for (int j = 0; j < BN; ++j) {
-                        const int64_t m = tm * BN + j;
+                        const int64_t m = cur_tm * BN + j;
                         if (m >= p.M) break;
                         int32_t* cell = wsl + j * SHERRY_TILE_ROWS + r;
                         const int32_t a32 = ptx::ld_cg_s32(cell);
