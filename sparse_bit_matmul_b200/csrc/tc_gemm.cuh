@@ -143,7 +143,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
-    volatile int* go_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);   // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -196,67 +195,75 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_holder;
 
     if (warp == kProducerWarp) {
-        if (lane == 0) {
-            int64_t issued = 0;
-            int64_t tile = u0 / p.Kc, c = u0 - (u0 / p.Kc) * p.Kc;
-            int64_t tm = tile / p.TN, tn = tile - (tile / p.TN) * p.TN;
-            int s = 0;
-            uint32_t ph = 0;
-            for (int64_t it = 0; it < n_it && !*abort_flag; ++it) {
-                if (!ptx::mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs)) {
-                    report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_PRODUCER);
-                    break;
-                }
+        // the whole warp runs the loop (converged); lane 0 issues the copies
+        int64_t issued = 0;
+        int64_t tile = u0 / p.Kc, c = u0 - (u0 / p.Kc) * p.Kc;
+        int64_t tm = tile / p.TN, tn = tile - (tile / p.TN) * p.TN;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int64_t it = 0; it < n_it; ++it) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            const bool ok = ptx::mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_PRODUCER);
+                break;
+            }
+            if (lane == 0) {
                 ptx::mbar_arrive_expect_tx(full_bar(s), (uint32_t)(kCodeStageBytes + C::kBStageBytes));
                 ptx::bulk_g2s(sbase + C::kOffCodes + (uint32_t)s * kCodeStageBytes,
                               p.wnative + (tn * p.Kc + c) * (int64_t)kCodeStageBytes, kCodeStageBytes,
                               full_bar(s));
                 ptx::tma_load_2d(sbase + (uint32_t)s * C::kBStageBytes, &xmap, (int32_t)(c * SHERRY_KCHUNK),
                                  (int32_t)(tm * BN), full_bar(s));
-                ++issued;
-                if (++s == C::kStages) { s = 0; ph ^= 1u; }
-                if (++c == p.Kc) {
-                    c = 0;
-                    if (++tn == p.TN) { tn = 0; ++tm; }
-                }
             }
-            // every copy issued has landed before the CTA may exit (in the
-            // normal flow the consumers already waited for all of them)
-            const int64_t from = issued > C::kStages ? issued - C::kStages : 0;
-            int ds = (int)(from % C::kStages);
-            uint32_t dph = (uint32_t)((from / C::kStages) & 1);
-            for (int64_t i = from; i < issued; ++i) {
-                if (!ptx::mbar_wait_bounded(full_bar(ds), dph, kWaitLimitNs)) {
-                    atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
-                    break;
-                }
-                if (++ds == C::kStages) { ds = 0; dph ^= 1u; }
+            __syncwarp();
+            ++issued;
+            if (++s == C::kStages) { s = 0; ph ^= 1u; }
+            if (++c == p.Kc) {
+                c = 0;
+                if (++tn == p.TN) { tn = 0; ++tm; }
             }
         }
+        // every copy issued has landed before the CTA may exit (in the
+        // normal flow the consumers already waited for all of them)
+        const int64_t from = issued > C::kStages ? issued - C::kStages : 0;
+        int ds = (int)(from % C::kStages);
+        uint32_t dph = (uint32_t)((from / C::kStages) & 1);
+        for (int64_t i = from; i < issued; ++i) {
+            const bool ok = ptx::mbar_wait_bounded(full_bar(ds), dph, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
+                break;
+            }
+            if (++ds == C::kStages) { ds = 0; dph ^= 1u; }
+        }
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            int64_t seg = 0;
-            int s = 0, a = 0, d = 0;
-            uint32_t sph = 0, aph = 0, dph = 0;
-            bool issued_any = false;
-            int64_t u = u0;
-            int64_t tile_end = (u0 / p.Kc + 1) * p.Kc;
-            while (u < u1 && !*abort_flag) {
-                const int64_t seg_end = tile_end < u1 ? tile_end : u1;
-                if (!ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs)) {
-                    report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
+        // the whole warp runs the loop (converged); lane 0 issues the MMAs
+        int s = 0, a = 0, d = 0;
+        uint32_t sph = 0, aph = 0, dph = 0;
+        bool issued_any = false;
+        int64_t u = u0;
+        int64_t tile_end = (u0 / p.Kc + 1) * p.Kc;
+        while (u < u1) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            const int64_t seg_end = tile_end < u1 ? tile_end : u1;
+            bool ok = ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
+            bool first = true;
+            for (; u < seg_end; ++u) {
+                ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs) &&
+                     ptx::mbar_wait_bounded(afull_bar(a), aph, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
                     break;
                 }
                 ptx::tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
-                bool first = true;
-                for (; u < seg_end; ++u) {
-                    if (!ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs) ||
-                        !ptx::mbar_wait_bounded(afull_bar(a), aph, kWaitLimitNs)) {
-                        report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
-                        break;
-                    }
-                    ptx::tc_fence_after();
+                if (lane == 0) {
                     const uint32_t a_tmem = tmem + (uint32_t)(C::kACol0 + a * 32);
                     const uint32_t b_addr = sbase + (uint32_t)s * C::kBStageBytes;
 #pragma unroll
@@ -264,25 +271,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::mma_i8_ts(d_tmem, a_tmem + 8u * ks, b_desc_sw128(b_addr + 32u * ks), C::kIdesc,
                                        (first && ks == 0) ? 0u : 1u);
                     }
-                    issued_any = true;
-                    first = false;
                     ptx::tc_commit(empty_bar(s));
                     ptx::tc_commit(aempty_bar(a));
-                    if (++s == C::kStages) { s = 0; sph ^= 1u; }
-                    if (++a == C::kAStages) { a = 0; aph ^= 1u; }
                 }
-                if (*abort_flag) break;
-                ptx::tc_commit(dfull_bar(d));
-                if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
-                tile_end += p.Kc;
-                ++seg;
+                __syncwarp();
+                issued_any = true;
+                first = false;
+                if (++s == C::kStages) { s = 0; sph ^= 1u; }
+                if (++a == C::kAStages) { a = 0; aph ^= 1u; }
             }
-            if (issued_any) {
-                // all MMAs of this thread complete before tensor memory is freed
-                ptx::tc_commit(drain_bar);
-                if (!ptx::mbar_wait_bounded(drain_bar, 0, kWaitLimitNs))
-                    atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
-            }
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            if (lane == 0) ptx::tc_commit(dfull_bar(d));
+            __syncwarp();
+            if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
+            tile_end += p.Kc;
+        }
+        if (issued_any) {
+            // all MMAs of this warp complete before tensor memory is freed
+            if (lane == 0) ptx::tc_commit(drain_bar);
+            __syncwarp();
+            const bool ok = ptx::mbar_wait_bounded(drain_bar, 0, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok) && lane == 0)
+                atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
         }
     } else if (warp >= kDecWarp0 && warp < kDecWarp0 + 4 * kDecGroups) {
         const int grp = (warp - kDecWarp0) / 4;
@@ -353,15 +363,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             u = seg_end;
             const int64_t n = tn * SHERRY_TILE_ROWS + r;
             const bool complete = (cb == 0 && ce == p.Kc);
-            // one thread waits, the decision is shared through a named barrier
-            // so that all 128 epilogue threads leave or stay together
-            if (etid == 0) {
-                bool ok = !*abort_flag && ptx::mbar_wait_bounded(dfull_bar(d), dph, kWaitLimitNs);
-                if (!ok && !*abort_flag) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_EPILOGUE);
-                go_flag[seg & 1] = ok ? 1 : 0;
+            // every epilogue thread waits; the AND over the 128 of them makes
+            // the leave-or-stay decision uniform
+            bool ok = !*abort_flag && ptx::mbar_wait_bounded(dfull_bar(d), dph, kWaitLimitNs);
+            ok = ptx::named_bar_and(1, 128, ok);
+            if (!ok) {
+                if (etid == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_EPILOGUE);
+                break;
             }
-            ptx::named_bar_sync(1, 128);
-            if (!go_flag[seg & 1]) break;
             ptx::tc_fence_after();
             const float al = (n < p.N) ? p.alpha[n] : 0.0f;
             int64_t slot = 0, nparts = 1;
@@ -407,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t old = atomicAdd(p.counters + slot, 1u);
                     *last_flag = (old == (uint32_t)(nparts - 1)) ? 1 : 0;
                 }
+                __syncwarp();
                 ptx::named_bar_sync(1, 128);
                 if (*last_flag) {
                     __threadfence();
@@ -423,11 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (etid == 0) atomicExch(p.counters + slot, 0u);
                 }
+                __syncwarp();
                 ptx::named_bar_sync(1, 128);
             }
         }
     }
 
+    __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
