@@ -161,6 +161,30 @@ int sherry_gemm_simt(const int8_t* x_i8, const float* x_scale, const void* Wnati
                      int64_t K, void* stream);
 
 /*
+ * sherry_gemm_noalloc -- device, asynchronous.  The same contraction and
+ * epilogue as sherry_gemm_acc, for callers that must not allocate device
+ * memory once they are running: programs whose device memory is handed out
+ * by their own pool sized at start-up, or whose request loop may not make
+ * the synchronising cudaMalloc/cudaFree calls.  (This entry point is an
+ * addition of this library; the Sherry page has no counterpart.)
+ * Instead of the per-device workspace of sherry_gemm, it uses a fixed
+ * scratch array compiled into the library: 2.6 MB, reserved on every GPU
+ * that loads the library until the process exits.  It therefore serves
+ * decode shapes only: M <= 32 tokens, otherwise SHERRY_ERR_UNSUPPORTED_SHAPE
+ * is returned before anything is launched.  It calls no cudaMalloc or
+ * cudaFree.  Each call first clears (cudaMemsetAsync on `stream`) the part
+ * of the scratch it uses.
+ * The first call on a device looks up the scratch's device address with that
+ * device current; make that first call before any stream capture.
+ * All calls share the one scratch array: calls that may overlap on the GPU
+ * (different streams without ordering between them) race and give wrong
+ * results.  Arguments as sherry_gemm_acc.
+ */
+int sherry_gemm_noalloc(const int8_t* x_i8, const float* x_scale, const void* Wnative,
+                        const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,
+                        int64_t K, void* stream);
+
+/*
  * sherry_last_device_status -- host, synchronous (copies one word from the
  * current device).  0 when no kernel of this library has reported a bounded
  * wait running out since the last reset; otherwise a nonzero code naming the

@@ -23,7 +23,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_NONFINITE, ERR_CUDA, ERR_DEVICE 
 ABI_SYMBOLS = (
     "sherry_status_string", "sherry_version", "sherry_packed_bytes", "sherry_native_bytes",
     "sherry_pack", "sherry_unpack", "sherry_repack", "sherry_quant_act", "sherry_gemm",
-    "sherry_gemm_acc", "sherry_gemm_simt", "sherry_last_device_status",
+    "sherry_gemm_acc", "sherry_gemm_simt", "sherry_gemm_noalloc", "sherry_last_device_status",
 )
 
 _lib = None
@@ -58,6 +58,7 @@ def load() -> ctypes.CDLL:
     L.sherry_gemm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_gemm_acc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_gemm_simt.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_gemm_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_last_device_status.argtypes = [c_int]
     for name in ABI_SYMBOLS:
         getattr(L, name).restype = getattr(L, name).restype or c_int
@@ -157,6 +158,8 @@ def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: boo
             rc = L.sherry_gemm_acc(*args)
     elif kernel == "simt":
         rc = L.sherry_gemm_simt(*args)
+    elif kernel == "noalloc":
+        rc = L.sherry_gemm_noalloc(*args)
     else:
         raise ValueError(kernel)
     _check(rc, f"sherry_gemm[{kernel}]")

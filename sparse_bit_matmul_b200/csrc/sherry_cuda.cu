@@ -319,6 +319,89 @@ int check_gemm_args(const int8_t* x, const float* xs, const void* wn, const floa
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for sherry_gemm_noalloc: the split-K partial sums and arrival
+// counters of at most kNoAllocMaxCtas CTAs for token tiles of up to
+// kNoAllocMaxBN tokens (M <= 32).  It lives in the library's own device
+// image, so it is reserved on every GPU that loads the library until exit.
+// ---------------------------------------------------------------------------
+constexpr int kNoAllocMaxCtas = 160;
+constexpr int kNoAllocMaxBN = 32;
+constexpr size_t kNoAllocAccWords = (size_t)kNoAllocMaxCtas * kNoAllocMaxBN * SHERRY_TILE_ROWS;
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocAccWords + kNoAllocMaxCtas];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+std::vector<int32_t*> g_noalloc_ptr;   // device address of g_noalloc_scratch, per device
+
+// Host code may not use g_noalloc_scratch's name as a device address: it is a
+// host-side stand-in.  The address is looked up once per device, with that
+// device current.
+int noalloc_scratch(int32_t** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SHERRY_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mutex);
+    if ((int)g_noalloc_ptr.size() <= dev) g_noalloc_ptr.resize(dev + 1, nullptr);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return SHERRY_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<int32_t*>(ptr);
+    }
+    *out = g_noalloc_ptr[dev];
+    return SHERRY_OK;
+}
+
+template <int BN>
+int launch_tc_noalloc(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y,
+                      int32_t* acc, int64_t M, int64_t N, int64_t K, cudaStream_t stream)
+{
+    using C = tc::Cfg<BN>;
+    static_assert(BN <= kNoAllocMaxBN, "token tile larger than the fixed scratch");
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != SHERRY_OK) return st;
+    int32_t* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != SHERRY_OK) return st;
+    tc::Params p;
+    p.wnative = static_cast<const uint8_t*>(wn);
+    p.alpha = alpha;
+    p.x_scale = xs;
+    p.y = y;
+    p.acc = acc;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.TM = (M + BN - 1) / BN;
+    p.TN = sherry_row_tiles(N);
+    p.Kc = sherry_k_chunks(K);
+    p.U = p.TM * p.TN * p.Kc;
+    const int64_t grid = std::min<int64_t>(std::min<int64_t>(di.sms, p.U), kNoAllocMaxCtas);
+    p.ws = scratch;
+    p.counters = reinterpret_cast<uint32_t*>(scratch + kNoAllocAccWords);
+    p.status = device_status_ptr();
+    if (!p.status) return SHERRY_ERR_CUDA;
+    // slots and counters this launch uses start at zero, whatever an earlier
+    // (possibly aborted) call left behind
+    if (cudaMemsetAsync(p.ws, 0, (size_t)grid * BN * SHERRY_TILE_ROWS * sizeof(int32_t), stream) != cudaSuccess ||
+        cudaMemsetAsync(p.counters, 0, (size_t)grid * sizeof(uint32_t), stream) != cudaSuccess)
+        return SHERRY_ERR_CUDA;
+    CUtensorMap map;
+    st = make_x_map(&map, x, M, K, BN);
+    if (st != SHERRY_OK) return st;
+    const int smem = std::max(C::kSmemBytes, 120 * 1024);
+    if (smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
+    if (cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+        return SHERRY_ERR_CUDA;
+    tc::sherry_gemm_tc_kernel<BN><<<(unsigned)grid, tc::kThreads, smem, stream>>>(map, p);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
 }  // namespace sherry
 
 using namespace sherry;
@@ -381,6 +464,17 @@ int sherry_gemm_simt(const int8_t* x_i8, const float* x_scale, const void* Wnati
     simt_gemm_kernel<<<grid, SHERRY_TILE_ROWS, 0, static_cast<cudaStream_t>(stream)>>>(
         x_i8, x_scale, static_cast<const uint32_t*>(Wnative), alpha, y, acc, M, N, K);
     return cuda_status(cudaGetLastError());
+}
+
+int sherry_gemm_noalloc(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha,
+                        float* y, int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
+    if (st != SHERRY_OK) return st;
+    if (M > kNoAllocMaxBN) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= 16) return launch_tc_noalloc<16>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    return launch_tc_noalloc<32>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
 }
 
 int sherry_last_device_status(int reset)
