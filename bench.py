@@ -48,7 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=["tc", "simt", "reference"], default="tc")
+    ap.add_argument("--impl", choices=["auto", "tc", "gemv", "simt", "reference"], default="auto",
+                    help="auto = sherry_gemm (GEMV kernel for M <= 4, tensor cores above)")
     ap.add_argument("--copies", type=int, default=32)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -369,7 +370,8 @@ def run_gpu(args, world, rank, local):
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak, "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-            "kernel": f"sherry_gemm_{kernel}", "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+            "kernel": "sherry_gemm_gemv (sherry_gemm at M=1)" if kernel == "auto" else f"sherry_gemm_{kernel}",
+            "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
             "avg_launch_us": round(gemm_launch_s * 1e6, 3),
             "algorithmic_bytes_per_launch": round(step_bytes / n_launch),
             "frac_of_8TBs_spec": round(achieved / 8000.0, 4),

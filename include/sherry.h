@@ -124,11 +124,16 @@ int sherry_repack(const uint8_t* codes_dev, int64_t N, int64_t K, void* native_d
 int sherry_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_i8, float* x_scale,
                      void* stream);
 
+/* Largest M that sherry_gemm runs on the decode GEMV kernel (for K <= 16384). */
+#define SHERRY_GEMV_MAX_M 4
+
 /*
  * sherry_gemm -- device, asynchronous.  y = epilogue(x_i8 . T^T) (sec. 2.2
- * steps 2-4): exact int32 accumulation on the tensor cores (tcgen05 kind::i8,
- * ternary weights decoded from the 5-bit codes into tensor memory), then
+ * steps 2-4): exact int32 accumulation, then
  * y[m][n] = (float)((float)acc * alpha[n]) * x_scale[m].
+ * M <= SHERRY_GEMV_MAX_M runs sherry_gemm_gemv (the page's activation-table
+ * lookup on the CUDA cores), larger M runs sherry_gemm_tc (tensor cores);
+ * both give identical results.
  *   x_i8     [in]  int8 [M][K], device memory, 16-byte aligned
  *   x_scale  [in]  fp32 [M], device memory
  *   Wnative  [in]  kernel-native codes from sherry_repack, device memory, 16-byte aligned
@@ -149,6 +154,35 @@ int sherry_gemm(const int8_t* x_i8, const float* x_scale, const void* Wnative,
 int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnative,
                     const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,
                     int64_t K, void* stream);
+
+/*
+ * sherry_gemm_tc -- device, asynchronous.  The contraction on the tensor
+ * cores for any M: the ternary weights are decoded from the 5-bit codes
+ * into tensor memory (one 32-bit cell per group of 4) and multiplied with
+ * tcgen05.mma kind::i8 against the int8 activations (TMA-loaded, 128-byte
+ * swizzle); K is split over all SMs with exact int32 partial sums in the
+ * per-device workspace.  Arguments as sherry_gemm_acc.
+ */
+int sherry_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* Wnative,
+                   const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,
+                   int64_t K, void* stream);
+
+/*
+ * sherry_gemm_gemv -- device, asynchronous.  Decode GEMV for M <= 
+ * SHERRY_GEMV_MAX_M tokens on the CUDA cores, following the page's
+ * inference scheme (sec. 2.2): per 4-element activation segment a table of
+ * its dot products with all 32 ternary groups is built in shared memory;
+ * each weight group then costs one table lookup and one add.  Launched with
+ * programmatic dependent launch (it may start before the previous kernel on
+ * the stream ends; it reads activations only after that kernel completed).
+ * The K-slices of a 128-row tile run as one thread-block cluster and are
+ * summed exactly through distributed shared memory (no workspace).  M > 4
+ * or K > 16384 returns SHERRY_ERR_UNSUPPORTED_SHAPE (sherry_gemm then uses
+ * the tensor-core kernel).  Arguments as sherry_gemm_acc.
+ */
+int sherry_gemm_gemv(const int8_t* x_i8, const float* x_scale, const void* Wnative,
+                     const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,
+                     int64_t K, void* stream);
 
 /*
  * sherry_gemm_simt -- device, asynchronous.  The same contraction and

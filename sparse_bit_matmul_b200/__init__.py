@@ -23,7 +23,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_NONFINITE, ERR_CUDA, ERR_DEVICE 
 ABI_SYMBOLS = (
     "sherry_status_string", "sherry_version", "sherry_packed_bytes", "sherry_native_bytes",
     "sherry_pack", "sherry_unpack", "sherry_repack", "sherry_quant_act", "sherry_gemm",
-    "sherry_gemm_acc", "sherry_gemm_simt", "sherry_gemm_noalloc", "sherry_last_device_status",
+    "sherry_gemm_acc", "sherry_gemm_tc", "sherry_gemm_gemv", "sherry_gemm_simt", "sherry_gemm_noalloc",
+    "sherry_last_device_status",
 )
 
 _lib = None
@@ -58,6 +59,8 @@ def load() -> ctypes.CDLL:
     L.sherry_gemm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_gemm_acc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_gemm_simt.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_gemm_tc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_gemm_gemv.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_gemm_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_last_device_status.argtypes = [c_int]
     for name in ABI_SYMBOLS:
@@ -139,10 +142,14 @@ def quant_act(x, out_q=None, out_s=None):
     return q, s
 
 
+GEMV_MAX_M = 4      # SHERRY_GEMV_MAX_M
+
+
 def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: bool = True,
-         kernel: str = "tc"):
+         kernel: str = "auto"):
     """y fp32 [M][N] (and optionally exact int32 acc) from int8 activations and
-    kernel-native codes.  kernel="simt" runs the CUDA-core comparison kernel."""
+    kernel-native codes.  kernel: "auto" (sherry_gemm: GEMV for M <= 4, tensor
+    cores above), "tc", "gemv", "simt" (comparison kernel) or "noalloc"."""
     import torch
     M, K = x_i8.shape
     y = None
@@ -151,11 +158,15 @@ def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: boo
     L = load()
     args = (_dptr(x_i8), _dptr(x_scale), _dptr(w_native), _dptr(alpha), _dptr(y), _dptr(acc), M, N, K,
             _stream(x_i8))
-    if kernel == "tc":
+    if kernel == "auto":
         if acc is None:
             rc = L.sherry_gemm(args[0], args[1], args[2], args[3], args[4], M, N, K, args[-1])
         else:
             rc = L.sherry_gemm_acc(*args)
+    elif kernel == "tc":
+        rc = L.sherry_gemm_tc(*args)
+    elif kernel == "gemv":
+        rc = L.sherry_gemm_gemv(*args)
     elif kernel == "simt":
         rc = L.sherry_gemm_simt(*args)
     elif kernel == "noalloc":

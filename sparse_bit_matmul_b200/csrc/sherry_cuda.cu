@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -12,6 +13,7 @@
 
 #include "sherry.h"
 #include "sherry_internal.h"
+#include "gemv.cuh"
 #include "tc_gemm.cuh"
 
 namespace sherry {
@@ -28,6 +30,8 @@ constexpr int kQuantThreads = 256;
 __global__ void __launch_bounds__(kQuantThreads)
     quant_act_kernel(const float* __restrict__ x, int64_t K, int8_t* __restrict__ q, float* __restrict__ scale)
 {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t m = blockIdx.x;
     const float4* xr = reinterpret_cast<const float4*>(x + m * K);
     char4* qr = reinterpret_cast<char4*>(q + m * K);
@@ -307,6 +311,79 @@ int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alp
     return cuda_status(cudaGetLastError());
 }
 
+// Launch with programmatic dependent launch: the kernel may start while the
+// previous kernel on the stream finishes; it orders itself with
+// griddepcontrol.wait before touching anything that kernel may write.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <int MT>
+int launch_gemv(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y, int32_t* acc,
+                int64_t M, int64_t N, int64_t K, cudaStream_t stream)
+{
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != SHERRY_OK) return st;
+    gemv::Params p;
+    p.wnative = static_cast<const uint8_t*>(wn);
+    p.x = x;
+    p.x_scale = xs;
+    p.alpha = alpha;
+    p.y = y;
+    p.acc = acc;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.TN = sherry_row_tiles(N);
+    p.Kc = sherry_k_chunks(K);
+    if (p.Kc > (int64_t)gemv::kMaxSL * gemv::kMaxNS || p.TN > 0x7fffffff) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    // K-slices per tile (the cluster size): enough for at most kMaxSL chunks
+    // per slice, more while the grid has fewer than two CTAs per SM
+    int NS = 1;
+    while (NS < gemv::kMaxNS && NS < p.Kc &&
+           ((p.Kc + NS - 1) / NS > gemv::kMaxSL || p.TN * NS < 2 * (int64_t)di.sms))
+        NS *= 2;
+    p.NS = NS;
+    p.SL = (int)((p.Kc + NS - 1) / NS);
+    p.status = device_status_ptr();
+    if (!p.status) return SHERRY_ERR_CUDA;
+    const int smem = gemv::smem_bytes(MT, p.SL);
+    if (smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(gemv::sherry_gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+        return SHERRY_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.TN, (unsigned)NS);
+    cfg.blockDim = dim3(gemv::kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = (unsigned)NS;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cuda_status(cudaLaunchKernelEx(&cfg, gemv::sherry_gemv_kernel<MT>, p));
+}
+
 int check_gemm_args(const int8_t* x, const float* xs, const void* wn, const float* alpha, const float* y,
                     const int32_t* acc, int64_t M, int64_t N, int64_t K)
 {
@@ -428,12 +505,22 @@ int sherry_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_i8, float* 
     if (M <= 0 || K <= 0) return SHERRY_ERR_INVALID_ARG;
     if (!sherry_shape_ok(M, 1, K)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x) || !aligned16(x_i8)) return SHERRY_ERR_INVALID_ARG;
-    quant_act_kernel<<<(unsigned)M, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(x, K, x_i8, x_scale);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch_pdl(quant_act_kernel, dim3((unsigned)M), dim3(kQuantThreads), 0,
+                                  static_cast<cudaStream_t>(stream), x, K, x_i8, x_scale));
 }
 
 int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,
                     int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
+    if (st != SHERRY_OK) return st;
+    if (M <= SHERRY_GEMV_MAX_M && sherry_k_chunks(K) <= (int64_t)gemv::kMaxSL * gemv::kMaxNS)
+        return sherry_gemm_gemv(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
+    return sherry_gemm_tc(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
+}
+
+int sherry_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,
+                   int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
 {
     int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
     if (st != SHERRY_OK) return st;
@@ -442,6 +529,19 @@ int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnativ
     if (M <= 32) return launch_tc<32>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
     if (M <= 64) return launch_tc<64>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
     return launch_tc<128>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+}
+
+int sherry_gemm_gemv(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,
+                     int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
+    if (st != SHERRY_OK) return st;
+    if (M > SHERRY_GEMV_MAX_M || sherry_k_chunks(K) > (int64_t)gemv::kMaxSL * gemv::kMaxNS)
+        return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 1) return launch_gemv<1>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    if (M == 2) return launch_gemv<2>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    return launch_gemv<4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
 }
 
 int sherry_gemm(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,

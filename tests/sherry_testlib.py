@@ -27,7 +27,7 @@ def upload_weights(W: np.ndarray, device="cuda"):
     return native, torch.from_numpy(alpha).to(device), codes, alpha
 
 
-def run_gpu(x: np.ndarray, native, alpha_dev, N: int, kernel="tc"):
+def run_gpu(x: np.ndarray, native, alpha_dev, N: int, kernel="auto"):
     """quant_act + gemm on the device; returns numpy (y, acc, q, s)."""
     import torch
     xd = torch.from_numpy(np.ascontiguousarray(x)).cuda()

@@ -68,12 +68,15 @@ def test_repack_layout(N, K):
 
 # ---------------------------------------------- small ragged shapes, full
 SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 512),
-         (64, 256, 1024), (100, 130, 4096), (129, 257, 160), (256, 512, 2048), (7, 1, 32)]
+         (64, 256, 1024), (100, 130, 4096), (129, 257, 160), (256, 512, 2048), (7, 1, 32),
+         (2, 4100, 1184), (4, 777, 14336), (1, 640, 9216), (2, 1, 32)]
 
 
-@pytest.mark.parametrize("kernel", ["tc", "simt"])
+@pytest.mark.parametrize("kernel", ["auto", "tc", "gemv", "simt"])
 @pytest.mark.parametrize("M,N,K", SMALL)
 def test_gemm_small_full(M, N, K, kernel):
+    if kernel == "gemv" and M > sbm.GEMV_MAX_M:
+        pytest.skip("the GEMV kernel serves M <= 4")
     W = synth.weights(0, 1, N, K, sigma=0.02)
     x = synth.activations(0, 1, M, K)
     y_o, acc_o, q_o, s_o, codes_o, alpha_o = oracle.reference(x, W)
@@ -102,7 +105,7 @@ def test_gemm_zero_token_and_repeat():
 
 
 # ----------------------------------------------- full-size configurations
-def _full_size_check(cfg, copy, M_list, K, N, int_mm=True):
+def _full_size_check(cfg, copy, M_list, K, N, int_mm=True, kernels=("auto",)):
     W = synth.config_weights(cfg, copy, K, N)
     native, alpha_d, codes, alpha = upload_weights(W)
     rows = rows_sample(N, seed=cfg * 7 + N)
@@ -113,11 +116,14 @@ def _full_size_check(cfg, copy, M_list, K, N, int_mm=True):
     for M in M_list:
         x = synth.config_activations(cfg, copy, M, K)
         q_o, s_o = oracle.quant_act(x)
-        y, acc, q, s = run_gpu(x, native, alpha_d, N)
-        assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
         acc_o = oracle.gemm(q_o, T_rows)
-        assert np.array_equal(acc[:, rows], acc_o)
-        assert_y_close(y[:, rows], oracle.epilogue(acc_o, a_rows, s_o))
+        for kern in kernels:
+            if kern == "gemv" and M > sbm.GEMV_MAX_M:
+                continue
+            y, acc, q, s = run_gpu(x, native, alpha_d, N, kern)
+            assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
+            assert np.array_equal(acc[:, rows], acc_o), kern
+            assert_y_close(y[:, rows], oracle.epilogue(acc_o, a_rows, s_o))
         if int_mm and M > 16:
             if T_full is None:
                 T_full, _ = oracle.quantise(W)
@@ -128,12 +134,12 @@ def _full_size_check(cfg, copy, M_list, K, N, int_mm=True):
 
 @pytest.mark.parametrize("K,N", synth.PROJ_SHAPES)
 def test_config1_decode_full_size(K, N):
-    _full_size_check(1, 0, [1], K, N)
+    _full_size_check(1, 0, [1], K, N, kernels=("auto", "tc"))
 
 
 @pytest.mark.parametrize("K,N", synth.PROJ_SHAPES)
 def test_config2_small_batch_full_size(K, N):
-    _full_size_check(2, 0, [4, 8, 16, 32], K, N)
+    _full_size_check(2, 0, [4, 8, 16, 32], K, N, kernels=("auto", "tc"))
 
 
 @pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096)])
@@ -142,7 +148,7 @@ def test_config3_prefill_full_size(K, N):
 
 
 def test_config4_heavy_tail_full_size():
-    W = _full_size_check(4, 0, [1, 128, 4096], 8192, 28672)
+    W = _full_size_check(4, 0, [1, 128, 4096], 8192, 28672, kernels=("auto", "tc"))
     T, _ = oracle.quantise(W)
     assert np.all(np.count_nonzero(T.reshape(28672, -1, 4), axis=2) == 3)
 
@@ -152,7 +158,7 @@ def test_config0_tiny_exact():
     x = synth.config_activations(0, 0, 1, 256)
     y_o, acc_o, *_ = oracle.reference(x, W)
     native, alpha_d, _, _ = upload_weights(W)
-    for kernel in ("tc", "simt"):
+    for kernel in ("auto", "tc", "gemv", "simt"):
         y, acc, _, _ = run_gpu(x, native, alpha_d, 128, kernel)
         assert np.array_equal(acc, acc_o)
         assert np.array_equal(y, y_o)
