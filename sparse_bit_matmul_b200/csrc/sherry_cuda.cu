@@ -244,6 +244,22 @@ int get_workspace(size_t bytes, cudaStream_t stream, void** out)
     return SHERRY_OK;
 }
 
+// fp32 y [M][N]: boxes of 128 rows n x 16 tokens m (no swizzle); needs rows
+// of whole 16-byte units (N % 4 == 0) and a 16-byte aligned base.
+int make_y_map(CUtensorMap* map, const float* y, int64_t M, int64_t N)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return SHERRY_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+    cuuint32_t box[2] = {SHERRY_TILE_ROWS, 16};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(y), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? SHERRY_OK : SHERRY_ERR_CUDA;
+}
+
 int make_x_map(CUtensorMap* map, const int8_t* x, int64_t M, int64_t K, int bn)
 {
     EncodeTiledFn enc = encode_fn();
@@ -265,11 +281,11 @@ unsigned* device_status_ptr()
     return static_cast<unsigned*>(p);
 }
 
-template <int BN>
+template <int BN, int SC>
 int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y, int32_t* acc,
               int64_t M, int64_t N, int64_t K, cudaStream_t stream)
 {
-    using C = tc::Cfg<BN>;
+    using C = tc::Cfg<BN, SC>;
     DeviceInfo di;
     int st = device_info(&di);
     if (st != SHERRY_OK) return st;
@@ -296,18 +312,21 @@ int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alp
     p.status = device_status_ptr();
     if (!p.status) return SHERRY_ERR_CUDA;
 
-    CUtensorMap map;
+    CUtensorMap map, ymap;
     st = make_x_map(&map, x, M, K, BN);
     if (st != SHERRY_OK) return st;
+    std::memset(&ymap, 0, sizeof(ymap));
+    p.y_tma = (y && N % 4 == 0 && aligned16(y)) ? 1 : 0;
+    if (p.y_tma && make_y_map(&ymap, y, M, N) != SHERRY_OK) p.y_tma = 0;
 
     // at least half of the SM's shared memory so that exactly one CTA (and
     // one 512-column tensor-memory allocation) lives on each SM
     const int smem = std::max(C::kSmemBytes, 120 * 1024);
     if (smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
-    cudaError_t e = cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN>,
+    cudaError_t e = cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN, SC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return SHERRY_ERR_CUDA;
-    tc::sherry_gemm_tc_kernel<BN><<<(unsigned)grid, tc::kThreads, smem, stream>>>(map, p);
+    tc::sherry_gemm_tc_kernel<BN, SC><<<(unsigned)grid, tc::kThreads, smem, stream>>>(map, ymap, p);
     return cuda_status(cudaGetLastError());
 }
 
@@ -430,11 +449,11 @@ int noalloc_scratch(int32_t** out)
     return SHERRY_OK;
 }
 
-template <int BN>
+template <int BN, int SC>
 int launch_tc_noalloc(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y,
                       int32_t* acc, int64_t M, int64_t N, int64_t K, cudaStream_t stream)
 {
-    using C = tc::Cfg<BN>;
+    using C = tc::Cfg<BN, SC>;
     static_assert(BN <= kNoAllocMaxBN, "token tile larger than the fixed scratch");
     DeviceInfo di;
     int st = device_info(&di);
@@ -465,15 +484,18 @@ int launch_tc_noalloc(const int8_t* x, const float* xs, const void* wn, const fl
     if (cudaMemsetAsync(p.ws, 0, (size_t)grid * BN * SHERRY_TILE_ROWS * sizeof(int32_t), stream) != cudaSuccess ||
         cudaMemsetAsync(p.counters, 0, (size_t)grid * sizeof(uint32_t), stream) != cudaSuccess)
         return SHERRY_ERR_CUDA;
-    CUtensorMap map;
+    CUtensorMap map, ymap;
     st = make_x_map(&map, x, M, K, BN);
     if (st != SHERRY_OK) return st;
+    std::memset(&ymap, 0, sizeof(ymap));
+    p.y_tma = (y && N % 4 == 0 && aligned16(y)) ? 1 : 0;
+    if (p.y_tma && make_y_map(&ymap, y, M, N) != SHERRY_OK) p.y_tma = 0;
     const int smem = std::max(C::kSmemBytes, 120 * 1024);
     if (smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
-    if (cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+    if (cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN, SC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return SHERRY_ERR_CUDA;
-    tc::sherry_gemm_tc_kernel<BN><<<(unsigned)grid, tc::kThreads, smem, stream>>>(map, p);
+    tc::sherry_gemm_tc_kernel<BN, SC><<<(unsigned)grid, tc::kThreads, smem, stream>>>(map, ymap, p);
     return cuda_status(cudaGetLastError());
 }
 
@@ -525,10 +547,10 @@ int sherry_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* Wnative
     int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
     if (st != SHERRY_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (M <= 16) return launch_tc<16>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
-    if (M <= 32) return launch_tc<32>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
-    if (M <= 64) return launch_tc<64>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
-    return launch_tc<128>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    if (M <= 16) return launch_tc<16, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    if (M <= 32) return launch_tc<32, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    if (M <= 64) return launch_tc<64, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    return launch_tc<128, 2>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
 }
 
 int sherry_gemm_gemv(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,
@@ -573,8 +595,8 @@ int sherry_gemm_noalloc(const int8_t* x_i8, const float* x_scale, const void* Wn
     if (st != SHERRY_OK) return st;
     if (M > kNoAllocMaxBN) return SHERRY_ERR_UNSUPPORTED_SHAPE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (M <= 16) return launch_tc_noalloc<16>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
-    return launch_tc_noalloc<32>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    if (M <= 16) return launch_tc_noalloc<16, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    return launch_tc_noalloc<32, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
 }
 
 int sherry_last_device_status(int reset)

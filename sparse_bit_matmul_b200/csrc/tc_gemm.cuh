@@ -26,9 +26,13 @@
 // the last contributor (an atomic counter) runs the epilogue and clears the
 // slot and counter, so the workspace is all zero between calls.
 //
+// A pipeline stage carries SC consecutive K chunks of one tile (one bulk copy
+// of SC * 2560 bytes of codes, SC 2D TMA boxes of activations, SC * 4 MMAs),
+// so that the fixed cost of a stage's barriers is paid once per SC chunks.
+//
 // Warp roles (576 threads):
-//   warp 0       producer: one bulk copy of 128 rows x 20 bytes of codes and
-//                one 2D TMA of the activation tile per K chunk
+//   warp 0       producer: per stage one bulk copy of the codes and one 2D
+//                TMA of the activation tile per chunk
 //   warp 1       TMEM allocation and MMA issue (one thread)
 //   warps 2-13   three decoder groups of four warps (each group covers the
 //                four TMEM lane quadrants), taking K chunks in turn
@@ -56,27 +60,38 @@ constexpr int kDecGroups = 3;
 constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;
 constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kTmemCols = 512;
-constexpr int kCodeStageBytes = SHERRY_CHUNK_BYTES_PER_TILE;   // 2560
+constexpr int kChunkCodeBytes = SHERRY_CHUNK_BYTES_PER_TILE;   // 2560
 constexpr uint64_t kWaitLimitNs = 2000000000ull;              // 2 s per wait
 
-template <int BN>
+template <int BN, int SC>
 struct Cfg {
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
-    static constexpr int kBStageBytes = BN * 128;
+    static_assert(SC >= 1 && SC <= 4, "SC");
+    static constexpr int kBChunkBytes = BN * 128;
+    static constexpr int kBStageBytes = SC * kBChunkBytes;
+    static constexpr int kCodeStageBytes = SC * kChunkCodeBytes;
     static constexpr int kStageBytes = kBStageBytes + kCodeStageBytes;
-    static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 24 ? 24 : kStagesRaw;
-    static constexpr int kDBufs = (2 * BN + 8 * 32 <= kTmemCols) ? 2 : 1;
-    static constexpr int kAStagesRaw = (kTmemCols - kDBufs * BN) / 32;
-    static constexpr int kAStages = kAStagesRaw > 12 ? 12 : kAStagesRaw;
+    static constexpr int kStagesRaw = (192 * 1024) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kACols = 32 * SC;                          // TMEM columns of one A stage
+    static constexpr int kDBufs = (2 * BN + 2 * kACols <= kTmemCols) ? 2 : 1;
+    static constexpr int kAStagesRaw = (kTmemCols - kDBufs * BN) / kACols;
+    static constexpr int kAStages = kAStagesRaw > 8 ? 8 : kAStagesRaw;
+    // A decoder group takes every kDecGroups-th stage.  Its phase-parity waits
+    // are exact only while the barrier it waits on is at most one phase
+    // behind: that holds when both rings are at least kDecGroups deep.
+    static_assert(kStages >= kDecGroups && kAStages >= kDecGroups, "pipeline rings shallower than decoder groups");
     static constexpr int kACol0 = kDBufs * BN;
     // shared memory: [B stages][code stages][barriers + misc]
     static constexpr int kOffCodes = kStages * kBStageBytes;
     static constexpr int kOffBars = kOffCodes + kStages * kCodeStageBytes;
     static constexpr int kNumBars = 2 * kStages + 2 * kAStages + 2 * kDBufs + 1;
     static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
-    static constexpr int kMiscBytes = 64;            // tmem holder, flags
-    static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;   // + alignment slack
+    static constexpr int kMiscBytes = 64 + 2 * BN * 4;   // tmem holder, flags, token scales [2][BN]
+    // output staging for TMA stores: two slices of [16 tokens][128 rows] fp32
+    static constexpr int kOffStaging = (kOffMisc + kMiscBytes + 127) & ~127;
+    static constexpr int kStagingBytes = 2 * 16 * 128 * 4;
+    static constexpr int kSmemBytes = kOffStaging + kStagingBytes + 1024;   // + alignment slack
     // instruction descriptor: s32 accumulate, signed int8 A and B, both
     // K-major, N = BN, M = 128
     static constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
@@ -95,6 +110,7 @@ struct Params {
     int64_t M, N, K;
     int64_t TM, TN, Kc;         // token tiles, row tiles, K chunks
     int64_t U;                  // total units TM*TN*Kc
+    int y_tma;                  // y rows 16-byte multiples: complete tiles leave through TMA stores
 };
 
 // CTA that owns unit u when U units are cut into G contiguous ranges
@@ -121,11 +137,44 @@ __device__ __forceinline__ void report(unsigned* status, volatile int* abort_fla
     *abort_flag = 1;
 }
 
-template <int BN>
+// The sequence of stages of one CTA: its unit range [u0, u1) cut at tile ends
+// into segments, each segment into stages of at most SC chunks.  Every role
+// walks this same sequence.
+template <int SC>
+struct StageWalk {
+    int64_t u, u1, Kc, tile, tile_end;
+    __device__ StageWalk(int64_t u0_, int64_t u1_, int64_t Kc_) : u(u0_), u1(u1_), Kc(Kc_)
+    {
+        tile = u0_ / Kc_;
+        tile_end = (tile + 1) * Kc_;
+    }
+    __device__ bool done() const { return u >= u1; }
+    __device__ int64_t seg_end() const { return tile_end < u1 ? tile_end : u1; }
+    __device__ int64_t chunk() const { return u - tile * Kc; }
+    __device__ int nch() const
+    {
+        const int64_t left = seg_end() - u;
+        return left < SC ? (int)left : SC;
+    }
+    // advance past the current stage; returns true when a segment ended
+    __device__ bool next()
+    {
+        u += nch();
+        if (u >= tile_end || u >= u1) {
+            ++tile;
+            tile_end += Kc;
+            return true;
+        }
+        return false;
+    }
+};
+
+template <int BN, int SC>
 __global__ void __launch_bounds__(kThreads, 1)
-    sherry_gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p)
+    sherry_gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap,
+                          const Params p)
 {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, SC>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ __align__(128) uint32_t table[32];
     // 1024-byte aligned start, computed by pointer arithmetic so that the
@@ -151,7 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t G = gridDim.x;
     const int64_t u0 = (p.U * (int64_t)blockIdx.x) / G;
     const int64_t u1 = (p.U * ((int64_t)blockIdx.x + 1)) / G;
-    const int64_t n_it = u1 - u0;
 
     if (threadIdx.x < 32) {
         // code -> four int8 weights of the group, byte i = position i
@@ -184,11 +232,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
+    __syncwarp();
     if (warp == kMmaWarp) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_holder), kTmemCols);
         ptx::tmem_relinquish();
     }
     if (threadIdx.x == 0) ptx::prefetch_tensormap(&xmap);
+    __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -197,30 +247,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kProducerWarp) {
         // the whole warp runs the loop (converged); lane 0 issues the copies
         int64_t issued = 0;
-        int64_t tile = u0 / p.Kc, c = u0 - (u0 / p.Kc) * p.Kc;
-        int64_t tm = tile / p.TN, tn = tile - (tile / p.TN) * p.TN;
+        int64_t tm = 0, tn = 0;
+        {
+            const int64_t tile = u0 / p.Kc;
+            tm = tile / p.TN;
+            tn = tile - tm * p.TN;
+        }
         int s = 0;
         uint32_t ph = 0;
-        for (int64_t it = 0; it < n_it; ++it) {
+        StageWalk<SC> wk(u0, u1, p.Kc);
+        while (!wk.done()) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             const bool ok = ptx::mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_PRODUCER);
                 break;
             }
+            const int nch = wk.nch();
+            const int64_t c = wk.chunk();
             if (lane == 0) {
-                ptx::mbar_arrive_expect_tx(full_bar(s), (uint32_t)(kCodeStageBytes + C::kBStageBytes));
-                ptx::bulk_g2s(sbase + C::kOffCodes + (uint32_t)s * kCodeStageBytes,
-                              p.wnative + (tn * p.Kc + c) * (int64_t)kCodeStageBytes, kCodeStageBytes,
-                              full_bar(s));
-                ptx::tma_load_2d(sbase + (uint32_t)s * C::kBStageBytes, &xmap, (int32_t)(c * SHERRY_KCHUNK),
-                                 (int32_t)(tm * BN), full_bar(s));
+                ptx::mbar_arrive_expect_tx(full_bar(s), (uint32_t)(nch * (kChunkCodeBytes + C::kBChunkBytes)));
+                ptx::bulk_g2s(sbase + C::kOffCodes + (uint32_t)s * C::kCodeStageBytes,
+                              p.wnative + (tn * p.Kc + c) * (int64_t)kChunkCodeBytes,
+                              (uint32_t)(nch * kChunkCodeBytes), full_bar(s));
+                for (int j = 0; j < nch; ++j)
+                    ptx::tma_load_2d(sbase + (uint32_t)(s * C::kBStageBytes + j * C::kBChunkBytes), &xmap,
+                                     (int32_t)((c + j) * SHERRY_KCHUNK), (int32_t)(tm * BN), full_bar(s));
             }
             __syncwarp();
             ++issued;
             if (++s == C::kStages) { s = 0; ph ^= 1u; }
-            if (++c == p.Kc) {
-                c = 0;
+            if (wk.next()) {
                 if (++tn == p.TN) { tn = 0; ++tm; }
             }
         }
@@ -241,50 +298,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the whole warp runs the loop (converged); lane 0 issues the MMAs
         int s = 0, a = 0, d = 0;
         uint32_t sph = 0, aph = 0, dph = 0;
-        bool issued_any = false;
-        int64_t u = u0;
-        int64_t tile_end = (u0 / p.Kc + 1) * p.Kc;
-        while (u < u1) {
+        bool issued_any = false, seg_start = true;
+        StageWalk<SC> wk(u0, u1, p.Kc);
+        while (!wk.done()) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            const int64_t seg_end = tile_end < u1 ? tile_end : u1;
-            bool ok = ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs);
+            bool ok = true;
+            if (seg_start) {
+                ok = ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
+                    break;
+                }
+            }
+            ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs) &&
+                 ptx::mbar_wait_bounded(afull_bar(a), aph, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
                 break;
             }
             ptx::tc_fence_after();
-            const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
-            bool first = true;
-            for (; u < seg_end; ++u) {
-                ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs) &&
-                     ptx::mbar_wait_bounded(afull_bar(a), aph, kWaitLimitNs);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
-                    break;
-                }
-                ptx::tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t a_tmem = tmem + (uint32_t)(C::kACol0 + a * 32);
-                    const uint32_t b_addr = sbase + (uint32_t)s * C::kBStageBytes;
+            const int nch = wk.nch();
+            if (lane == 0) {
+                const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
+                const uint32_t a_tmem = tmem + (uint32_t)(C::kACol0 + a * C::kACols);
+                // descriptor of the stage's first K step; later steps only add
+                // to the start-address field (16-byte units)
+                const uint64_t desc0 = b_desc_sw128(sbase + (uint32_t)s * C::kBStageBytes);
+                const uint32_t acc0 = seg_start ? 0u : 1u;
+                if (nch == SC) {
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        ptx::mma_i8_ts(d_tmem, a_tmem + 8u * ks, b_desc_sw128(b_addr + 32u * ks), C::kIdesc,
-                                       (first && ks == 0) ? 0u : 1u);
-                    }
-                    ptx::tc_commit(empty_bar(s));
-                    ptx::tc_commit(aempty_bar(a));
+                    for (int j = 0; j < SC; ++j)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            ptx::mma_i8_ts(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
+                                           desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
+                                           (j == 0 && ks == 0) ? acc0 : 1u);
+                } else {
+                    for (int j = 0; j < nch; ++j)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            ptx::mma_i8_ts(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
+                                           desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
+                                           (j == 0 && ks == 0) ? acc0 : 1u);
                 }
-                __syncwarp();
-                issued_any = true;
-                first = false;
-                if (++s == C::kStages) { s = 0; sph ^= 1u; }
-                if (++a == C::kAStages) { a = 0; aph ^= 1u; }
+                ptx::tc_commit(empty_bar(s));
+                ptx::tc_commit(aempty_bar(a));
             }
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            if (lane == 0) ptx::tc_commit(dfull_bar(d));
             __syncwarp();
-            if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
-            tile_end += p.Kc;
+            issued_any = true;
+            seg_start = false;
+            if (++s == C::kStages) { s = 0; sph ^= 1u; }
+            if (++a == C::kAStages) { a = 0; aph ^= 1u; }
+            if (wk.next()) {
+                if (lane == 0) ptx::tc_commit(dfull_bar(d));
+                __syncwarp();
+                if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
+                seg_start = true;
+            }
         }
         if (issued_any) {
             // all MMAs of this warp complete before tensor memory is freed
@@ -300,50 +370,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = quad * 32 + lane;          // row within the 128-row tile
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         const uint8_t* tbl = reinterpret_cast<const uint8_t*>(table);
-        // stage and phase of iteration it = grp, grp + G, grp + 2G, ...
-        int s = grp % C::kStages, a = grp % C::kAStages;
-        uint32_t sph = (uint32_t)((grp / C::kStages) & 1), aph = (uint32_t)((grp / C::kAStages) & 1);
-        for (int64_t it = grp; it < n_it; it += kDecGroups) {
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            bool ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
-                break;
-            }
-            const uint32_t* codes =
-                reinterpret_cast<const uint32_t*>(smem + C::kOffCodes + s * kCodeStageBytes);
-            uint32_t w[SHERRY_CHUNK_WORDS];
+        int s = 0, a = 0;
+        uint32_t sph = 0, aph = 0;
+        int turn = 0;                               // iteration index modulo kDecGroups
+        StageWalk<SC> wk(u0, u1, p.Kc);
+        for (; !wk.done(); wk.next(), turn = (turn + 1 == kDecGroups) ? 0 : turn + 1) {
+            const int nch = wk.nch();
+            const bool mine = turn == grp;
+            if (mine) {
+                if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                bool ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
+                    break;
+                }
+                const uint32_t* codes =
+                    reinterpret_cast<const uint32_t*>(smem + C::kOffCodes + s * C::kCodeStageBytes);
+                uint32_t w[SC][SHERRY_CHUNK_WORDS];
 #pragma unroll
-            for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) w[j] = codes[j * SHERRY_TILE_ROWS + row];
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(empty_bar(s));
-            uint32_t a_vals[32];
+                for (int j = 0; j < SC; ++j)
 #pragma unroll
-            for (int g = 0; g < 32; ++g) {
-                // byte offset of the group's table entry: code * 4
-                const int bit = 5 * g, wi = bit >> 5, off = bit & 31;
-                uint32_t v;
-                if (off == 0) v = w[wi] << 2;
-                else if (off == 1) v = w[wi] << 1;
-                else if (off <= 27) v = w[wi] >> (off - 2);
-                else v = __funnelshift_r(w[wi], w[wi + 1], off - 2);
-                a_vals[g] = *reinterpret_cast<const uint32_t*>(tbl + (v & 0x7Cu));
+                    for (int k = 0; k < SHERRY_CHUNK_WORDS; ++k)
+                        w[j][k] = (j < nch) ? codes[(j * SHERRY_CHUNK_WORDS + k) * SHERRY_TILE_ROWS + row] : 0u;
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(empty_bar(s));
+                ok = ptx::mbar_wait_bounded(aempty_bar(a), aph ^ 1u, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
+                    break;
+                }
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < SC; ++j) {
+                    if (j >= nch) break;
+                    uint32_t a_vals[32];
+#pragma unroll
+                    for (int g = 0; g < 32; ++g) {
+                        // byte offset of the group's table entry: code * 4
+                        const int bit = 5 * g, wi = bit >> 5, off = bit & 31;
+                        uint32_t v;
+                        if (off == 0) v = w[j][wi] << 2;
+                        else if (off == 1) v = w[j][wi] << 1;
+                        else if (off <= 27) v = w[j][wi] >> (off - 2);
+                        else v = __funnelshift_r(w[j][wi], w[j][wi + 1], off - 2);
+                        a_vals[g] = *reinterpret_cast<const uint32_t*>(tbl + (v & 0x7Cu));
+                    }
+                    ptx::tmem_st_32x32b_x32(lane_base + (uint32_t)(C::kACol0 + a * C::kACols + 32 * j), a_vals);
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(afull_bar(a));
             }
-            ok = ptx::mbar_wait_bounded(aempty_bar(a), aph ^ 1u, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
-                break;
-            }
-            ptx::tc_fence_after();
-            ptx::tmem_st_32x32b_x32(lane_base + (uint32_t)(C::kACol0 + a * 32), a_vals);
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(afull_bar(a));
-            s += kDecGroups;
-            if (s >= C::kStages) { s -= C::kStages; sph ^= 1u; }
-            a += kDecGroups;
-            if (a >= C::kAStages) { a -= C::kAStages; aph ^= 1u; }
+            if (++s == C::kStages) { s = 0; sph ^= 1u; }
+            if (++a == C::kAStages) { a = 0; aph ^= 1u; }
         }
     } else if (warp >= kEpiWarp0) {
         const int quad = warp & 3;
@@ -356,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int64_t tm = tile / p.TN, tn = tile - (tile / p.TN) * p.TN;
         int d = 0;
         uint32_t dph = 0;
+        uint32_t stage_slice = 0;                  // output slices staged so far
         while (u < u1) {
             const int64_t cb = u - tile * p.Kc;
             const int64_t seg_end = (tile + 1) * p.Kc < u1 ? (tile + 1) * p.Kc : u1;
@@ -363,6 +444,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             u = seg_end;
             const int64_t n = tn * SHERRY_TILE_ROWS + r;
             const bool complete = (cb == 0 && ce == p.Kc);
+            // the tile's token scales and this row's alpha do not depend on
+            // the MMAs: fetch them into shared memory (double-buffered by
+            // segment) before waiting for the accumulators
+            float* sc_s = reinterpret_cast<float*>(smem + C::kOffMisc + 64) + (seg & 1) * BN;
+            for (int i = etid; i < BN; i += 128) {
+                const int64_t m = tm * BN + i;
+                sc_s[i] = (m < p.M) ? __ldg(p.x_scale + m) : 0.0f;
+            }
+            const float al = (n < p.N) ? __ldg(p.alpha + n) : 0.0f;
             // every epilogue thread waits; the AND over the 128 of them makes
             // the leave-or-stay decision uniform
             bool ok = !*abort_flag && ptx::mbar_wait_bounded(dfull_bar(d), dph, kWaitLimitNs);
@@ -372,7 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             ptx::tc_fence_after();
-            const float al = (n < p.N) ? p.alpha[n] : 0.0f;
             int64_t slot = 0, nparts = 1;
             if (!complete) {
                 const int64_t bf = owner_of(tile * p.Kc, p.U, G);
@@ -381,11 +470,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 nparts = bl - bf + 1;
             }
             int32_t* wsl = p.ws + slot * (int64_t)BN * SHERRY_TILE_ROWS;
+            const bool via_tma = complete && p.y_tma && p.y && !p.acc;
 #pragma unroll 1
             for (int j0 = 0; j0 < BN; j0 += 16) {
+                if (via_tma && tm * BN + j0 >= p.M) break;     // rows past M: nothing to store
                 uint32_t v[16];
+                if (via_tma) {
+                    // staging buffer of this slice is free once the store
+                    // issued two slices ago has read it
+                    if (etid == 0) ptx::bulk_wait_group_read<1>();
+                    ptx::named_bar_sync(1, 128);
+                }
                 ptx::tmem_ld_32x32b_x16(lane_base + (uint32_t)(d * BN + j0), v);
                 ptx::tmem_wait_ld();
+                if (via_tma) {
+                    float* stg = reinterpret_cast<float*>(smem + C::kOffStaging) + (stage_slice & 1) * (16 * 128);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj)
+                        stg[jj * 128 + r] = __fmul_rn(__fmul_rn((float)(int32_t)v[jj], al), sc_s[j0 + jj]);
+                    ptx::fence_proxy_async_smem();
+                    ptx::named_bar_sync(1, 128);
+                    if (etid == 0) {
+                        ptx::tma_store_2d(&ymap, (int32_t)(tn * SHERRY_TILE_ROWS), (int32_t)(tm * BN + j0),
+                                          ptx::smem_u32(stg));
+                        ptx::bulk_commit_group();
+                    }
+                    ++stage_slice;
+                    continue;
+                }
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     const int64_t m = tm * BN + j0 + jj;
@@ -394,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (complete) {
                         if (n < p.N) {
                             if (p.acc) p.acc[m * p.N + n] = a32;
-                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, al), p.x_scale[m]);
+                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, al), sc_s[j0 + jj]);
                         }
                     } else {
                         ptx::red_add_s32(wsl + (j0 + jj) * SHERRY_TILE_ROWS + r, a32);
@@ -428,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *cell = 0;
                         if (n < p.N) {
                             if (p.acc) p.acc[m * p.N + n] = a32;
-                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, al), p.x_scale[m]);
+                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, al), sc_s[j]);
                         }
                     }
                     if (etid == 0) atomicExch(p.counters + slot, 0u);
@@ -437,6 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::named_bar_sync(1, 128);
             }
         }
+        // shared memory stays valid until every TMA store has read it
+        if (etid == 0) ptx::bulk_wait_group<0>();
     }
 
     __syncwarp();

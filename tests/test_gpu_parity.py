@@ -69,7 +69,8 @@ def test_repack_layout(N, K):
 # ---------------------------------------------- small ragged shapes, full
 SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 512),
          (64, 256, 1024), (100, 130, 4096), (129, 257, 160), (256, 512, 2048), (7, 1, 32),
-         (2, 4100, 1184), (4, 777, 14336), (1, 640, 9216), (2, 1, 32)]
+         (2, 4100, 1184), (4, 777, 14336), (1, 640, 9216), (2, 1, 32), (300, 1024, 2048),
+         (200, 388, 4096), (130, 8192, 256)]
 
 
 @pytest.mark.parametrize("kernel", ["auto", "tc", "gemv", "simt"])
@@ -86,6 +87,9 @@ def test_gemm_small_full(M, N, K, kernel):
     assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
     assert np.array_equal(acc, acc_o)
     assert_y_close(y, y_o)
+    if kernel in ("auto", "tc"):
+        y2, _, _, _ = run_gpu(x, native, alpha_d, N, kernel, with_acc=False)
+        assert_y_close(y2, y_o)
 
 
 def test_gemm_zero_token_and_repeat():
@@ -123,7 +127,10 @@ def _full_size_check(cfg, copy, M_list, K, N, int_mm=True, kernels=("auto",)):
             y, acc, q, s = run_gpu(x, native, alpha_d, N, kern)
             assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
             assert np.array_equal(acc[:, rows], acc_o), kern
-            assert_y_close(y[:, rows], oracle.epilogue(acc_o, a_rows, s_o))
+            y_ref_rows = oracle.epilogue(acc_o, a_rows, s_o)
+            assert_y_close(y[:, rows], y_ref_rows)
+            y2, _, _, _ = run_gpu(x, native, alpha_d, N, kern, with_acc=False)
+            assert np.array_equal(y2, y), kern          # y-only path (TMA stores) gives the same y
         if int_mm and M > 16:
             if T_full is None:
                 T_full, _ = oracle.quantise(W)
