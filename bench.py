@@ -46,14 +46,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["auto", "tc", "gemv", "simt", "reference"], default="auto",
                     help="auto = sherry_gemm (GEMV kernel for M <= 4, tensor cores above)")
     ap.add_argument("--copies", type=int, default=32)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["decode", "prefill"], default=None,
+                    help="run a few launches of one layer shape (K=4096, N=14336; M=1 or 2048) "
+                         "and exit: the target of the committed ncu captures")
     return ap.parse_args(argv)
 
 
@@ -81,9 +84,10 @@ def host_cores() -> int:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms; only the
+    samples whose timestamps fall inside the timed window are summarised."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -91,43 +95,70 @@ class ClockSampler:
         self.gpu_index = gpu_index
         self.proc = None
         self.lines = []
+        self.thread = None
+        self.window = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
 
     def start(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.gpu_index)],
+                 "-lms", "50", "-i", str(self.gpu_index)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t_end = time.time() + 5.0
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
+
+    def mark(self, begin: float, end: float):
+        self.window = (begin, end)
 
     def stop(self):
         if self.proc is None:
             return None
+        time.sleep(0.12)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], None, set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        from datetime import datetime
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+        for line in self.lines:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[5:9]):
+        if not rows:
+            return None
+        inside = rows
+        if self.window is not None:
+            b, e = self.window
+            inside = [r for r in rows if b <= r[0] <= e] or \
+                     [min(rows, key=lambda r: abs(r[0] - 0.5 * (b + e)))]
+        reasons = set()
+        for r in inside:
+            for nm, v in zip(names, r[3]):
                 if v.lower().startswith("active"):
                     reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": inside[-1][2],
+                "reasons": sorted(reasons), "samples": len(inside),
+                "window_s": round(self.window[1] - self.window[0], 3) if self.window else None}
 
 
 # ------------------------------------------------------------- distributed
@@ -277,7 +308,7 @@ def capture(fn, warm: int = 2):
     return g
 
 
-def time_graph(g, steps: int, warmup: int, world: int):
+def time_graph(g, steps: int, warmup: int, world: int, sampler=None):
     import torch
     for _ in range(warmup):
         g.replay()
@@ -285,11 +316,15 @@ def time_graph(g, steps: int, warmup: int, world: int):
     barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
     e0.record()
     for _ in range(steps):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
+    w1 = time.time()
+    if sampler is not None:
+        sampler.mark(w0, w1)
     barrier(world)
     return e0.elapsed_time(e1) / 1e3
 
@@ -334,7 +369,7 @@ def run_gpu(args, world, rank, local):
 
     sampler = ClockSampler(local)
     sampler.start()
-    t_step = time_graph(g_step, args.steps, args.warmup, world)
+    t_step = time_graph(g_step, args.steps, args.warmup, world, sampler)
     clocks = sampler.stop()
     t_step = max_over_ranks(t_step, world)
     t_gemm = max_over_ranks(time_graph(g_gemm, args.steps, args.warmup, world), world)
@@ -348,7 +383,8 @@ def run_gpu(args, world, rank, local):
     n_launch = len(layers)
     gemm_launch_s = t_gemm / (args.steps * n_launch)
     achieved = step_bytes / (t_gemm / args.steps) / 1e9
-    traffic = load_traffic()
+    traffic = load_traffic("sherry_gemv_kernel<1>" if kernel in ("auto", "gemv") else f"sherry_gemm_{kernel}",
+                           step_bytes / n_launch)
     h2d = sum(L["x"].numel() * 4 for L in layers)
     d2h = sum(L["y"].numel() * 4 for L in layers)
 
@@ -392,13 +428,19 @@ def run_gpu(args, world, rank, local):
     return out
 
 
-def load_traffic():
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if current."""
+def load_traffic(kernel: str, avg_algorithmic_bytes: float):
+    """DRAM bytes per launch of the dominant kernel: the committed ncu capture
+    (profiles/traffic.json, one launch of one layer shape) scaled to the
+    average launch of the step by algorithmic bytes.  None when the capture
+    is not of the kernel this run times."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return d.get("decode_gemm_bytes_per_launch")
+        e = d.get(kernel)
+        if not e:
+            return None
+        return round(e["dram_bytes"] / e["algorithmic_bytes"] * avg_algorithmic_bytes)
     except Exception:
         return None
 
@@ -462,11 +504,56 @@ def extras(args, layers, kernel, peaks, peak_src, world):
     res["prefill_M2048"] = pre
     res["int8_peak_tops"] = {"value": round(int8_peak, 1),
                              "source": f"{peak_src} bf16_tflops x nominal int8/bf16 ratio 2"}
+    # practical dense INT8 tensor throughput of the library GEMM on this machine
+    a = torch.randint(-127, 128, (8192, 8192), dtype=torch.int8, device="cuda")
+    b = torch.randint(-127, 128, (8192, 8192), dtype=torch.int8, device="cuda").t()
+    for _ in range(3):
+        torch._int_mm(a, b)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(10):
+        torch._int_mm(a, b)
+    e1.record()
+    torch.cuda.synchronize()
+    lib_tops = 2.0 * 8192 ** 3 * 10 / (e0.elapsed_time(e1) / 1e3) / 1e12
+    res["int8_library_gemm_tops"] = {"value": round(lib_tops, 1), "how": "torch._int_mm 8192^3, 10 launches"}
+    for v in pre.values():
+        v["frac_of_library_int8"] = round(v["int_tops_dense_equiv"] / lib_tops, 4)
     return res
+
+
+def profile_case(args):
+    """A few launches of one layer shape, small enough for a full ncu capture."""
+    import torch
+    import sparse_bit_matmul_b200 as sbm
+    import synth
+    torch.cuda.set_device(0)
+    sbm.load()
+    M, K, N = (1, 4096, 14336) if args.profile_case == "decode" else (2048, 4096, 14336)
+    copies = 8 if M == 1 else 1
+    layers = []
+    for c in range(copies):
+        codes, alpha = sbm.pack(synth.config_weights(1 if M == 1 else 3, c, K, N))
+        layers.append((sbm.repack(torch.from_numpy(codes).cuda(), N, K), torch.from_numpy(alpha).cuda()))
+    x = torch.from_numpy(synth.config_activations(1 if M == 1 else 3, 0, M, K)).cuda()
+    q, s = sbm.quant_act(x)
+    y = torch.empty((M, N), device="cuda")
+    kernel = "auto" if args.impl == "reference" else args.impl
+    for _ in range(4):
+        for nat, al in layers:
+            sbm.gemm(q, s, nat, al, N, out=y, kernel=kernel)
+    torch.cuda.synchronize()
+    status = sbm.last_device_status()
+    print(json.dumps({"profile_case": args.profile_case, "M": M, "K": K, "N": N, "copies": copies,
+                      "launches": 4 * copies, "kernel": kernel, "device_status": status}))
+    return 0 if status == 0 else 1
 
 
 def main(argv=None):
     args = parse_args(argv)
+    if args.profile_case:
+        return profile_case(args)
     world, rank, local = dist_setup(args.gpus, need_cuda=(args.impl != "reference"))
     try:
         if args.impl == "reference":
