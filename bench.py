@@ -48,8 +48,9 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--impl", choices=["auto", "tc", "gemv", "simt", "reference"], default="auto",
-                    help="auto = sherry_gemm (GEMV kernel for M <= 4, tensor cores above)")
+    ap.add_argument("--impl", choices=["auto", "decode", "tc", "gemv", "simt", "reference"], default="auto",
+                    help="auto = sherry_linear (quantiser fused into the decode GEMM); others = "
+                         "sherry_quant_act + that GEMM kernel")
     ap.add_argument("--copies", type=int, default=32)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -342,29 +343,47 @@ def run_gpu(args, world, rank, local):
     step_bytes = sum(algorithmic_bytes(M, L["K"], L["N"]) for L in layers)
     code_bytes = sum(L["N"] * L["K"] * 5 // 32 for L in layers)
 
-    def step():
-        for L in layers:
+    # auto: sherry_linear, one fused launch per layer call (quantiser + GEMM);
+    # otherwise sherry_quant_act + the named GEMM kernel, two launches
+    fused = kernel == "auto"
+
+    def layer(L):
+        if fused:
+            sbm.linear(L["x"], L["native"], L["alpha"], L["N"], out=L["y"])
+        else:
             sbm.quant_act(L["x"], L["q"], L["s"])
             sbm.gemm(L["q"], L["s"], L["native"], L["alpha"], L["N"], out=L["y"], kernel=kernel)
 
+    def step():
+        for L in layers:
+            layer(L)
+
     def gemm_only():
         for L in layers:
-            sbm.gemm(L["q"], L["s"], L["native"], L["alpha"], L["N"], out=L["y"], kernel=kernel)
+            sbm.gemm(L["q"], L["s"], L["native"], L["alpha"], L["N"], out=L["y"],
+                     kernel="auto" if fused else kernel)
 
     def quant_only():
         for L in layers:
             sbm.quant_act(L["x"], L["q"], L["s"])
 
+    def two_launch_step():
+        for L in layers:
+            sbm.quant_act(L["x"], L["q"], L["s"])
+            sbm.gemm(L["q"], L["s"], L["native"], L["alpha"], L["N"], out=L["y"])
+
     def e2e_step():
         for L in layers:
             L["x"].copy_(L["x_host"], non_blocking=True)
-            sbm.quant_act(L["x"], L["q"], L["s"])
-            sbm.gemm(L["q"], L["s"], L["native"], L["alpha"], L["N"], out=L["y"], kernel=kernel)
+            layer(L)
             L["y_host"].copy_(L["y"], non_blocking=True)
 
+    for L in layers:                  # q, s for the GEMM-only graphs
+        sbm.quant_act(L["x"], L["q"], L["s"])
     g_step = capture(step)
     g_gemm = capture(gemm_only)
     g_quant = capture(quant_only)
+    g_two = capture(two_launch_step) if fused else None
     g_e2e = capture(e2e_step)
 
     sampler = ClockSampler(local)
@@ -374,6 +393,7 @@ def run_gpu(args, world, rank, local):
     t_step = max_over_ranks(t_step, world)
     t_gemm = max_over_ranks(time_graph(g_gemm, args.steps, args.warmup, world), world)
     t_quant = max_over_ranks(time_graph(g_quant, args.steps, args.warmup, world), world)
+    t_two = max_over_ranks(time_graph(g_two, args.steps, args.warmup, world), world) if fused else None
     t_e2e = max_over_ranks(time_graph(g_e2e, args.steps, args.warmup, world), world)
     assert sbm.last_device_status() == 0, "a kernel reported a bounded wait running out"
 
@@ -381,10 +401,12 @@ def run_gpu(args, world, rank, local):
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     value = step_bytes * world * args.steps / t_step / 1e9
     n_launch = len(layers)
-    gemm_launch_s = t_gemm / (args.steps * n_launch)
-    achieved = step_bytes / (t_gemm / args.steps) / 1e9
-    traffic = load_traffic("sherry_gemv_kernel<1>" if kernel in ("auto", "gemv") else f"sherry_gemm_{kernel}",
-                           step_bytes / n_launch)
+    # the dominant kernel: the fused kernel is the whole step; otherwise the GEMM
+    t_dom = t_step if fused else t_gemm
+    dom_launch_s = t_dom / (args.steps * n_launch)
+    achieved = step_bytes / (t_dom / args.steps) / 1e9
+    dom_name = "sherry_decode_kernel<1,fused>" if fused else f"sherry_gemm_{kernel}"
+    traffic = load_traffic(dom_name, step_bytes / n_launch)
     h2d = sum(L["x"].numel() * 4 for L in layers)
     d2h = sum(L["y"].numel() * 4 for L in layers)
 
@@ -400,27 +422,34 @@ def run_gpu(args, world, rank, local):
             "M": 1, "copies_per_gpu": args.copies, "layers_per_step": n_launch,
             "bytes_per_step": step_bytes, "packed_weight_bytes_per_step": code_bytes,
             "l2": "inputs larger than L2: %.0f MB of packed weights per step vs 126 MB L2" % (code_bytes / 1e6),
-            "launch": "one CUDA graph per step (quant_act + GEMM per layer)", "kernel": kernel,
+            "launch": ("one CUDA graph per step: sherry_linear per layer (activation quantiser fused "
+                       "into the decode GEMM, one launch)") if fused else
+                      "one CUDA graph per step: sherry_quant_act + GEMM per layer", "kernel": kernel,
             "parallelism": f"replicas x{world} (independent layer copies per GPU)",
         },
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak, "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-            "kernel": "sherry_gemm_gemv (sherry_gemm at M=1)" if kernel == "auto" else f"sherry_gemm_{kernel}",
+            "kernel": dom_name,
             "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
-            "avg_launch_us": round(gemm_launch_s * 1e6, 3),
+            "avg_launch_us": round(dom_launch_s * 1e6, 3),
             "algorithmic_bytes_per_launch": round(step_bytes / n_launch),
             "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
         },
-        "quant_act": {"avg_launch_us": round(t_quant / (args.steps * n_launch) * 1e6, 3)},
+        "separate_kernels": {
+            "quant_act_avg_launch_us": round(t_quant / (args.steps * n_launch) * 1e6, 3),
+            "gemm_avg_launch_us": round(t_gemm / (args.steps * n_launch) * 1e6, 3),
+            "gemm_gbs": round(step_bytes / (t_gemm / args.steps) / 1e9, 2),
+            "two_launch_step_gbs": (round(step_bytes * args.steps / t_two / 1e9, 2) if fused else None),
+        },
         "e2e": {"value": round(step_bytes * world * args.steps / t_e2e / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "path": "pinned host x -> H2D -> sherry_quant_act -> sherry_gemm -> D2H y, per layer, "
-                        "in one CUDA graph per step"},
-        "gpu_launches": 2 * n_launch * args.steps,
+                "path": ("pinned host x -> H2D -> " + ("sherry_linear" if fused else "sherry_quant_act -> "
+                         f"sherry_gemm[{kernel}]") + " -> D2H y, per layer, in one CUDA graph per step")},
+        "gpu_launches": (1 if fused else 2) * n_launch * args.steps,
         "clocks": clocks,
     }
-    del g_step, g_gemm, g_quant, g_e2e
+    del g_step, g_gemm, g_quant, g_two, g_e2e
     if not args.no_extras:
         out["extra"] = extras(args, layers, kernel, peaks, peak_src, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -453,18 +482,19 @@ def extras(args, layers, kernel, peaks, peak_src, world):
     # small-batch decode on the same weights (M = 4, 8, 16, 32)
     small = {}
     for M in (4, 8, 16, 32):
-        xs = {}
+        xs, xf = {}, {}
         for L in layers:
             key = L["K"]
             if key not in xs:
-                xq = torch.from_numpy(synth.config_activations(2, 0, M, key)).cuda()
-                q, s = sbm.quant_act(xq)
-                xs[key] = (q, s)
+                xf[key] = torch.from_numpy(synth.config_activations(2, 0, M, key)).cuda()
+                xs[key] = sbm.quant_act(xf[key])
         ys = {L["N"]: torch.empty((M, L["N"]), device="cuda") for L in layers}
 
         def fn():
             for L in layers:
                 q, s = xs[L["K"]]
+                if kernel == "auto":
+                    sbm.quant_act(xf[L["K"]], q, s)
                 sbm.gemm(q, s, L["native"], L["alpha"], L["N"], out=ys[L["N"]], kernel=kernel)
         g = capture(fn)
         t = max_over_ranks(time_graph(g, max(3, args.steps // 4), 2, world), world)
@@ -472,6 +502,9 @@ def extras(args, layers, kernel, peaks, peak_src, world):
         small[str(M)] = round(nb * max(3, args.steps // 4) / t / 1e9, 2)
         del g
     res["small_batch_decode_gbs"] = small
+    res["small_batch_step"] = ("sherry_quant_act + sherry_gemm (decode kernel for M <= 8, tensor cores above) "
+                               "per layer call"
+                               if kernel == "auto" else f"GEMM kernel {kernel} only")
     # prefill GEMM, M = 2048 (L2 flushed between timed launches)
     int8_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * NOMINAL_INT8_OVER_BF16
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
@@ -542,7 +575,10 @@ def profile_case(args):
     kernel = "auto" if args.impl == "reference" else args.impl
     for _ in range(4):
         for nat, al in layers:
-            sbm.gemm(q, s, nat, al, N, out=y, kernel=kernel)
+            if kernel == "auto" and M == 1:
+                sbm.linear(x, nat, al, N, out=y)
+            else:
+                sbm.gemm(q, s, nat, al, N, out=y, kernel=kernel)
     torch.cuda.synchronize()
     status = sbm.last_device_status()
     print(json.dumps({"profile_case": args.profile_case, "M": M, "K": K, "N": N, "copies": copies,

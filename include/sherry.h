@@ -101,7 +101,11 @@ int sherry_unpack(const uint8_t* codes, int64_t N, int64_t K, int8_t* T);
  * sherry_repack -- device, asynchronous on `stream`.  Rearranges a canonical
  * code stream already copied to the device into the kernel-native layout
  * (same codes, tile-interleaved so that 128 consecutive rows of one 128-wide
- * K chunk are one contiguous 2560-byte block).
+ * K chunk are one contiguous 2560-byte block).  Inside a block, word j
+ * (canonical bytes [20c+4j, 20c+4j+4) of the row, little endian) of row r
+ * sits at 32-bit index 128 j + ((r + 8 j) mod 128): five word planes, plane
+ * j rotated by 8 j rows so that the kernels' shared-memory reads of it are
+ * free of bank conflicts.
  *   codes_dev  [in]  uint8 [N][5K/32], device memory
  *   native_dev [out] sherry_native_bytes(N, K) bytes, device memory, 16-byte aligned
  * Padding bytes are written as zero.
@@ -124,16 +128,21 @@ int sherry_repack(const uint8_t* codes_dev, int64_t N, int64_t K, void* native_d
 int sherry_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_i8, float* x_scale,
                      void* stream);
 
-/* Largest M that sherry_gemm runs on the decode GEMV kernel (for K <= 16384). */
+/* Largest M of the table-lookup GEMV kernel, sherry_gemm_gemv. */
 #define SHERRY_GEMV_MAX_M 4
+/* Largest M of the decode kernel, sherry_gemm_decode. */
+#define SHERRY_DECODE_MAX_M 8
+/* Largest M for which sherry_linear is a single fused launch. */
+#define SHERRY_LINEAR_FUSED_MAX_M 4
 
 /*
  * sherry_gemm -- device, asynchronous.  y = epilogue(x_i8 . T^T) (sec. 2.2
  * steps 2-4): exact int32 accumulation, then
  * y[m][n] = (float)((float)acc * alpha[n]) * x_scale[m].
- * M <= SHERRY_GEMV_MAX_M runs sherry_gemm_gemv (the page's activation-table
- * lookup on the CUDA cores), larger M runs sherry_gemm_tc (tensor cores);
- * both give identical results.
+ * M <= SHERRY_DECODE_MAX_M runs sherry_gemm_decode (when a CTA's share of
+ * the codes fits in shared memory, i.e. K up to about 600000 weights), any
+ * other shape sherry_gemm_tc (tensor cores); all kernels give identical
+ * results.
  *   x_i8     [in]  int8 [M][K], device memory, 16-byte aligned
  *   x_scale  [in]  fp32 [M], device memory
  *   Wnative  [in]  kernel-native codes from sherry_repack, device memory, 16-byte aligned
@@ -168,6 +177,56 @@ int sherry_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* Wnative
                    int64_t K, void* stream);
 
 /*
+ * sherry_gemm_decode -- device, asynchronous.  The decode kernel for
+ * M <= SHERRY_DECODE_MAX_M tokens, on the CUDA cores.  One CTA per SM owns a
+ * balanced range of whole output rows over the full K: its codes are
+ * streamed into shared memory, each 5-bit code becomes four int8 weights in
+ * {-1,0,+1} through a 32-entry table, and dp4a adds them against the int8
+ * activations; partial sums of a row never leave the CTA (no workspace, no
+ * atomics).  Launched with programmatic dependent launch: the weight copy
+ * starts before the previous kernel on the stream ends; activations are
+ * read only after it completed, so Wnative and alpha must not be written by
+ * the kernel launched just before on the same stream unless that kernel
+ * ends without triggering its dependents early (every ordinary kernel, and
+ * sherry_repack, does so).  Returns SHERRY_ERR_UNSUPPORTED_SHAPE for M > 8
+ * or when one row's codes do not fit in shared memory.  Arguments as
+ * sherry_gemm_acc.
+ */
+int sherry_gemm_decode(const int8_t* x_i8, const float* x_scale, const void* Wnative,
+                       const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,
+                       int64_t K, void* stream);
+
+/*
+ * sherry_linear -- device, asynchronous.  The whole online step of the page
+ * (sec. 2.2 steps 1-4) from fp32 activations: the sherry_quant_act rule
+ * followed by the sherry_gemm contraction and epilogue, with bit-identical
+ * results.  For M <= SHERRY_LINEAR_FUSED_MAX_M it is one launch of the
+ * decode kernel that also quantises (every CTA reads the whole activation
+ * rows, takes their absmax and quantises them into its shared memory).
+ * Other shapes run sherry_quant_act into a per-device buffer of the library
+ * (allocated on first use, grown with a stream synchronisation) and then
+ * sherry_gemm.
+ *   x        [in]  fp32 [M][K], device memory, 16-byte aligned
+ *   Wnative  [in]  kernel-native codes, device memory, 16-byte aligned
+ *   alpha    [in]  fp32 [N], device memory
+ *   y        [out] fp32 [M][N], device memory
+ * Concurrency as sherry_gemm.  (The page describes these steps as one
+ * inference pass; the single entry point is this library's.)
+ */
+int sherry_linear(const float* x, const void* Wnative, const float* alpha, float* y,
+                  int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * sherry_linear_ex -- as sherry_linear, with optional outputs: acc int32
+ * [M][N], and x_i8 int8 [M][K] (16-byte aligned) with x_scale fp32 [M], the
+ * quantised activations (both or neither; when given they are also used
+ * instead of the library's buffer).  y may be NULL when acc is given.
+ */
+int sherry_linear_ex(const float* x, const void* Wnative, const float* alpha, float* y,
+                     int32_t* acc, int8_t* x_i8, float* x_scale, int64_t M, int64_t N,
+                     int64_t K, void* stream);
+
+/*
  * sherry_gemm_gemv -- device, asynchronous.  Decode GEMV for M <= 
  * SHERRY_GEMV_MAX_M tokens on the CUDA cores, following the page's
  * inference scheme (sec. 2.2): per 4-element activation segment a table of
@@ -177,8 +236,9 @@ int sherry_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* Wnative
  * the stream ends; it reads activations only after that kernel completed).
  * The K-slices of a 128-row tile run as one thread-block cluster and are
  * summed exactly through distributed shared memory (no workspace).  M > 4
- * or K > 16384 returns SHERRY_ERR_UNSUPPORTED_SHAPE (sherry_gemm then uses
- * the tensor-core kernel).  Arguments as sherry_gemm_acc.
+ * or K > 16384 returns SHERRY_ERR_UNSUPPORTED_SHAPE.  sherry_gemm does not
+ * dispatch to it; it is the page's own scheme, kept for comparison with
+ * sherry_gemm_decode.  Arguments as sherry_gemm_acc.
  */
 int sherry_gemm_gemv(const int8_t* x_i8, const float* x_scale, const void* Wnative,
                      const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,

@@ -24,7 +24,7 @@ ABI_SYMBOLS = (
     "sherry_status_string", "sherry_version", "sherry_packed_bytes", "sherry_native_bytes",
     "sherry_pack", "sherry_unpack", "sherry_repack", "sherry_quant_act", "sherry_gemm",
     "sherry_gemm_acc", "sherry_gemm_tc", "sherry_gemm_gemv", "sherry_gemm_simt", "sherry_gemm_noalloc",
-    "sherry_last_device_status",
+    "sherry_gemm_decode", "sherry_linear", "sherry_linear_ex", "sherry_last_device_status",
 )
 
 _lib = None
@@ -62,6 +62,9 @@ def load() -> ctypes.CDLL:
     L.sherry_gemm_tc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_gemm_gemv.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_gemm_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_gemm_decode.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_linear.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_linear_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_last_device_status.argtypes = [c_int]
     for name in ABI_SYMBOLS:
         getattr(L, name).restype = getattr(L, name).restype or c_int
@@ -143,13 +146,16 @@ def quant_act(x, out_q=None, out_s=None):
 
 
 GEMV_MAX_M = 4      # SHERRY_GEMV_MAX_M
+DECODE_MAX_M = 8    # SHERRY_DECODE_MAX_M
+LINEAR_FUSED_MAX_M = 4   # SHERRY_LINEAR_FUSED_MAX_M
 
 
 def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: bool = True,
          kernel: str = "auto"):
     """y fp32 [M][N] (and optionally exact int32 acc) from int8 activations and
-    kernel-native codes.  kernel: "auto" (sherry_gemm: GEMV for M <= 4, tensor
-    cores above), "tc", "gemv", "simt" (comparison kernel) or "noalloc"."""
+    kernel-native codes.  kernel: "auto" (sherry_gemm: the decode kernel
+    for M <= 8, tensor cores above), "decode", "tc", "gemv" (the page's
+    table lookup), "simt" (comparison kernel) or "noalloc"."""
     import torch
     M, K = x_i8.shape
     y = None
@@ -171,9 +177,31 @@ def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: boo
         rc = L.sherry_gemm_simt(*args)
     elif kernel == "noalloc":
         rc = L.sherry_gemm_noalloc(*args)
+    elif kernel == "decode":
+        rc = L.sherry_gemm_decode(*args)
     else:
         raise ValueError(kernel)
     _check(rc, f"sherry_gemm[{kernel}]")
+    return y
+
+
+def linear(x, w_native, alpha, N: int, out=None, acc=None, out_q=None, out_s=None, want_y: bool = True):
+    """y fp32 [M][N] straight from fp32 activations x [M][K] (sherry_linear:
+    quantiser + GEMM, one launch for M <= 4).  Optional acc int32 [M][N] and
+    out_q int8 [M][K] / out_s fp32 [M] receive the exact accumulators and the
+    quantised activations."""
+    import torch
+    M, K = x.shape
+    y = None
+    if want_y:
+        y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
+    L = load()
+    if acc is None and out_q is None and out_s is None:
+        rc = L.sherry_linear(_dptr(x), _dptr(w_native), _dptr(alpha), _dptr(y), M, N, K, _stream(x))
+    else:
+        rc = L.sherry_linear_ex(_dptr(x), _dptr(w_native), _dptr(alpha), _dptr(y), _dptr(acc), _dptr(out_q),
+                                _dptr(out_s), M, N, K, _stream(x))
+    _check(rc, "sherry_linear")
     return y
 
 
@@ -187,7 +215,7 @@ class PackedLinear:
     ``PackedLinear.from_weights(W)`` packs on the host (sherry_pack), copies
     the canonical codes and alpha to the device and repacks them into the
     kernel-native layout.  ``forward(x)`` quantises the activations and runs
-    the GEMM; both are asynchronous on the current stream.
+    the GEMM (sherry_linear), asynchronously on the current stream.
     """
 
     def __init__(self, w_native, alpha, N: int, K: int):
@@ -208,5 +236,4 @@ class PackedLinear:
         return cls(w_native, torch.from_numpy(alpha).to(device), N, K)
 
     def forward(self, x, out=None):
-        q, s = quant_act(x)
-        return gemm(q, s, self.w_native, self.alpha, self.N, out=out)
+        return linear(x, self.w_native, self.alpha, self.N, out=out)

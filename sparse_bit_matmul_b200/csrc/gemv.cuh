@@ -57,28 +57,6 @@ struct Params {
     int SL, NS;                 // chunks per slice, slices per tile (cluster size)
 };
 
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents()
-{
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire()
-{
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Adds v to the int32 at `local_addr`'s offset in the shared memory of CTA `cta`
-// of the cluster.
-__device__ __forceinline__ void red_cluster_add_s32(uint32_t local_addr, uint32_t cta, int32_t v)
-{
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(cta));
-    asm volatile("red.shared::cluster.add.s32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
-}
-
 // Shared memory of one CTA for MT tokens and SL chunks per slice: the tables
 // (token stride fixed so that the token offset is an immediate), the codes,
 // the partial sums [2][MT][128] int32 (the second half doubles as the receive
@@ -147,10 +125,10 @@ __global__ void __launch_bounds__(kThreads)
     for (int i = threadIdx.x; i < MT * 128; i += kThreads) recv[i] = 0;
     if (p.NS > 1) {
         __syncthreads();
-        cluster_arrive_release();
+        ptx::cluster_arrive_release();
     }
-    pdl_launch_dependents();
-    pdl_wait();
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
 
     // tables of this K-slice: one (token, group) per thread and step
     const int G = nch * 32;
@@ -184,7 +162,7 @@ __global__ void __launch_bounds__(kThreads)
         uint32_t w[SHERRY_CHUNK_WORDS];
 #pragma unroll
         for (int k = 0; k < SHERRY_CHUNK_WORDS; ++k)
-            w[k] = codes[(j * SHERRY_CHUNK_WORDS + k) * SHERRY_TILE_ROWS + row];
+            w[k] = codes[j * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS) + sherry_word_pos(k, row)];
         const uint32_t base = lut_base + (uint32_t)j * 2048u;   // 64-byte aligned
 #pragma unroll
         for (int g = 0; g < 32; ++g) {
@@ -217,17 +195,17 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
             for (int m = 0; m < MT; ++m) recv[m * 128 + row] = acc[m];
         } else {
-            cluster_wait_acquire();             // every peer has zeroed its receive buffer
+            ptx::cluster_wait_acquire();             // every peer has zeroed its receive buffer
             const uint32_t owner = (uint32_t)(row / rows);
 #pragma unroll
-            for (int m = 0; m < MT; ++m) red_cluster_add_s32(ptx::smem_u32(recv + m * 128 + row), owner, acc[m]);
+            for (int m = 0; m < MT; ++m) ptx::red_cluster_add_s32(ptx::smem_u32(recv + m * 128 + row), owner, acc[m]);
         }
     } else if (p.NS > 1) {
-        cluster_wait_acquire();
+        ptx::cluster_wait_acquire();
     }
     if (p.NS > 1) {
-        cluster_arrive_release();               // partial sums sent
-        cluster_wait_acquire();                 // ... and received from every peer
+        ptx::cluster_arrive_release();               // partial sums sent
+        ptx::cluster_wait_acquire();                 // ... and received from every peer
     } else {
         __syncthreads();
     }

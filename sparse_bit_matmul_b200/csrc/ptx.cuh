@@ -234,5 +234,64 @@ __device__ __forceinline__ int32_t ld_cg_s32(const int32_t* p)
     return v;
 }
 
+
+// ---- programmatic dependent launch ------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- thread-block clusters ----------------------------------------------------
+__device__ __forceinline__ void cluster_arrive_release()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of `local_addr`'s counterpart in the shared memory of cluster CTA `cta`.
+__device__ __forceinline__ uint32_t mapa(uint32_t local_addr, uint32_t cta)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(cta));
+    return remote;
+}
+// Adds v to the int32 at `local_addr`'s offset in the shared memory of CTA `cta`.
+__device__ __forceinline__ void red_cluster_add_s32(uint32_t local_addr, uint32_t cta, int32_t v)
+{
+    asm volatile("red.shared::cluster.add.s32 [%0], %1;" ::"r"(mapa(local_addr, cta)), "r"(v) : "memory");
+}
+// Shared load the compiler may schedule freely (no side effects declared).
+__device__ __forceinline__ uint32_t lds_u32_nv(uint32_t addr)
+{
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_u64(uint32_t addr)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
 }  // namespace ptx
 }  // namespace sherry

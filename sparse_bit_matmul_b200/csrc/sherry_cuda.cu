@@ -14,6 +14,8 @@
 #include "sherry.h"
 #include "sherry_internal.h"
 #include "gemv.cuh"
+#include "decode.cuh"
+#include "quant.cuh"
 #include "tc_gemm.cuh"
 
 namespace sherry {
@@ -23,7 +25,7 @@ __device__ unsigned g_device_status = 0;
 // ---------------------------------------------------------------------------
 // Activation quantiser: one CTA per token.  a = max |x| (exact), s = a / 127
 // (IEEE fp32 division), q = clamp(rint(x / s), -127, 127) with rint rounding
-// half to even; a == 0 gives s = 0 and q = 0.
+// half to even; a == 0 gives s = 0 and q = 0 (the arithmetic of quant.cuh).
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 256;
 
@@ -34,10 +36,11 @@ __global__ void __launch_bounds__(kQuantThreads)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t m = blockIdx.x;
     const float4* xr = reinterpret_cast<const float4*>(x + m * K);
-    char4* qr = reinterpret_cast<char4*>(q + m * K);
+    int8_t* qr = q + m * K;
     const int64_t K4 = K / 4;
 
     float a = 0.0f;
+#pragma unroll 4
     for (int64_t i = threadIdx.x; i < K4; i += kQuantThreads) {
         const float4 v = xr[i];
         a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
@@ -51,21 +54,11 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
     for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, warp_max[w]);
 
-    const float s = __fdiv_rn(a, 127.0f);
-    if (threadIdx.x == 0) scale[m] = (a == 0.0f) ? 0.0f : s;
-    for (int64_t i = threadIdx.x; i < K4; i += kQuantThreads) {
-        char4 o = make_char4(0, 0, 0, 0);
-        if (a != 0.0f) {
-            const float4 v = xr[i];
-            auto qz = [s](float f) -> signed char {
-                int r = __float2int_rn(__fdiv_rn(f, s));
-                r = r > 127 ? 127 : (r < -127 ? -127 : r);
-                return (signed char)r;
-            };
-            o = make_char4(qz(v.x), qz(v.y), qz(v.z), qz(v.w));
-        }
-        qr[i] = o;
-    }
+    const quant::Scale sc = quant::make_scale(a);
+    if (threadIdx.x == 0) scale[m] = sc.s;
+    uint32_t* qw = reinterpret_cast<uint32_t*>(qr);
+#pragma unroll 4
+    for (int64_t i = threadIdx.x; i < K4; i += kQuantThreads) qw[i] = quant::quantise4(xr[i], sc);
 }
 
 // ---------------------------------------------------------------------------
@@ -78,8 +71,8 @@ __global__ void repack_kernel(const uint8_t* __restrict__ codes, int64_t N, int6
     const int64_t Kc = sherry_k_chunks(K);
     for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total_words;
          idx += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = idx % SHERRY_TILE_ROWS;
         const int64_t j = (idx / SHERRY_TILE_ROWS) % SHERRY_CHUNK_WORDS;
+        const int64_t r = (idx - 8 * j) & (SHERRY_TILE_ROWS - 1);    // position idx % 128 holds row r
         const int64_t c = (idx / (SHERRY_TILE_ROWS * SHERRY_CHUNK_WORDS)) % Kc;
         const int64_t t = idx / (SHERRY_TILE_ROWS * SHERRY_CHUNK_WORDS * Kc);
         const int64_t n = t * SHERRY_TILE_ROWS + r;
@@ -129,7 +122,7 @@ __global__ void __launch_bounds__(SHERRY_TILE_ROWS)
         const uint32_t* blk = wn + (t * Kc + c) * (SHERRY_TILE_ROWS * SHERRY_CHUNK_WORDS);
         uint32_t w[SHERRY_CHUNK_WORDS + 1];
 #pragma unroll
-        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) w[j] = blk[j * SHERRY_TILE_ROWS + r];
+        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) w[j] = blk[sherry_word_pos(j, r)];
         w[SHERRY_CHUNK_WORDS] = 0;
         for (int g = 0; g < 32; ++g) {
             const int64_t k = c * SHERRY_KCHUNK + 4 * g;
@@ -403,6 +396,99 @@ int launch_gemv(const int8_t* x, const float* xs, const void* wn, const float* a
     return cuda_status(cudaLaunchKernelEx(&cfg, gemv::sherry_gemv_kernel<MT>, p));
 }
 
+// Work split of the decode kernel: G CTAs of at most R rows (one per SM
+// unless the codes of R rows would not fit the shared-memory budget), P
+// K-parts of CPT chunks per row, R * P <= kMaxThreads.  False if even one
+// row does not fit.
+struct DecodePlan {
+    int G, R, P, CPT, threads, smem;
+};
+
+bool decode_plan(int64_t N, int64_t Kc, int64_t M, int sms, DecodePlan* out)
+{
+    int64_t G = std::min<int64_t>(sms, N);
+    for (int iter = 0; iter < 64; ++iter) {
+        const int64_t R = (N + G - 1) / G;
+        if (R > decode::kMaxThreads) {
+            G = (N + decode::kMaxThreads - 1) / decode::kMaxThreads;
+            continue;
+        }
+        int64_t P = std::max<int64_t>(1, std::min<int64_t>(Kc, decode::kMaxThreads / R));
+        const int64_t CPT = (Kc + P - 1) / P;
+        P = (Kc + CPT - 1) / CPT;
+        const int64_t smem = decode::smem_bytes((int)M, (int)P, (int)R, Kc);
+        if (smem <= decode::kSmemBudget) {
+            if (G > 0x7fffffff) return false;
+            out->G = (int)G;
+            out->R = (int)R;
+            out->P = (int)P;
+            out->CPT = (int)CPT;
+            out->threads = (int)((R * P + 31) / 32 * 32);
+            out->smem = (int)smem;
+            return true;
+        }
+        if (R == 1) return false;
+        G = (N + R / 2 - 1) / (R / 2);          // halve the rows per CTA
+    }
+    return false;
+}
+
+template <int MT, bool FUSED>
+int launch_decode(const decode::Params& p0, cudaStream_t stream)
+{
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != SHERRY_OK) return st;
+    decode::Params p = p0;
+    p.Kc = sherry_k_chunks(p.K);
+    if (p.M > MT) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    DecodePlan pl;
+    if (!decode_plan(p.N, p.Kc, p.M, di.sms, &pl)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    p.G = pl.G;
+    p.R = pl.R;
+    p.P = pl.P;
+    p.CPT = pl.CPT;
+    if (pl.smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [&] {
+        attr_err = cudaFuncSetAttribute(decode::sherry_decode_kernel<MT, FUSED>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, decode::kSmemBudget);
+    });
+    if (attr_err != cudaSuccess) return SHERRY_ERR_CUDA;
+    return cuda_status(launch_pdl(decode::sherry_decode_kernel<MT, FUSED>, dim3((unsigned)pl.G),
+                                  dim3((unsigned)pl.threads), (size_t)pl.smem, stream, p));
+}
+
+// Per-device buffer for the int8 activations and scales of sherry_linear
+// when the caller passes none and the fused kernel does not apply.
+std::vector<Workspace> g_act;
+
+int get_act_buffer(size_t bytes, cudaStream_t stream, void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SHERRY_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((int)g_act.size() <= dev) g_act.resize(dev + 1);
+    Workspace& w = g_act[dev];
+    if (w.bytes < bytes) {
+        if (w.ptr) {
+            if (cudaStreamSynchronize(stream) != cudaSuccess) return SHERRY_ERR_CUDA;
+            cudaFree(w.ptr);
+            w.ptr = nullptr;
+            w.bytes = 0;
+        }
+        size_t nb = std::max<size_t>(bytes, size_t(1) << 20);
+        if (cudaMalloc(&w.ptr, nb) != cudaSuccess) {
+            w.ptr = nullptr;
+            return SHERRY_ERR_CUDA;
+        }
+        w.bytes = nb;
+    }
+    *out = w.ptr;
+    return SHERRY_OK;
+}
+
 int check_gemm_args(const int8_t* x, const float* xs, const void* wn, const float* alpha, const float* y,
                     const int32_t* acc, int64_t M, int64_t N, int64_t K)
 {
@@ -536,9 +622,89 @@ int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnativ
 {
     int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
     if (st != SHERRY_OK) return st;
-    if (M <= SHERRY_GEMV_MAX_M && sherry_k_chunks(K) <= (int64_t)gemv::kMaxSL * gemv::kMaxNS)
-        return sherry_gemm_gemv(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
+    if (M <= SHERRY_DECODE_MAX_M) {
+        DeviceInfo di;
+        st = device_info(&di);
+        if (st != SHERRY_OK) return st;
+        DecodePlan pl;
+        if (decode_plan(N, sherry_k_chunks(K), M, di.sms, &pl))
+            return sherry_gemm_decode(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
+    }
     return sherry_gemm_tc(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
+}
+
+int sherry_gemm_decode(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha,
+                       float* y, int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
+    if (st != SHERRY_OK) return st;
+    if (M > SHERRY_DECODE_MAX_M) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    decode::Params p = {};
+    p.wnative = static_cast<const uint8_t*>(Wnative);
+    p.xq = x_i8;
+    p.x_scale = x_scale;
+    p.alpha = alpha;
+    p.y = y;
+    p.acc = acc;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 1) return launch_decode<1, false>(p, s);
+    if (M == 2) return launch_decode<2, false>(p, s);
+    if (M <= 4) return launch_decode<4, false>(p, s);
+    return launch_decode<8, false>(p, s);
+}
+
+int sherry_linear_ex(const float* x, const void* Wnative, const float* alpha, float* y, int32_t* acc,
+                     int8_t* x_i8, float* x_scale, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    if (!x || !Wnative || !alpha || (!y && !acc)) return SHERRY_ERR_INVALID_ARG;
+    if ((x_i8 == nullptr) != (x_scale == nullptr)) return SHERRY_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return SHERRY_ERR_INVALID_ARG;
+    if (!sherry_shape_ok(M, N, K)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(Wnative) || (x_i8 && !aligned16(x_i8))) return SHERRY_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= SHERRY_LINEAR_FUSED_MAX_M) {
+        DeviceInfo di;
+        int st = device_info(&di);
+        if (st != SHERRY_OK) return st;
+        DecodePlan pl;
+        if (decode_plan(N, sherry_k_chunks(K), M, di.sms, &pl)) {
+            decode::Params p = {};
+            p.wnative = static_cast<const uint8_t*>(Wnative);
+            p.x = x;
+            p.xq_out = x_i8;
+            p.xs_out = x_scale;
+            p.alpha = alpha;
+            p.y = y;
+            p.acc = acc;
+            p.M = M;
+            p.N = N;
+            p.K = K;
+            if (M == 1) return launch_decode<1, true>(p, s);
+            if (M == 2) return launch_decode<2, true>(p, s);
+            return launch_decode<4, true>(p, s);
+        }
+    }
+    if (!x_i8) {
+        void* buf = nullptr;
+        const size_t qbytes = ((size_t)M * (size_t)K + 255) & ~size_t(255);
+        int st = get_act_buffer(qbytes + (size_t)M * sizeof(float), s, &buf);
+        if (st != SHERRY_OK) return st;
+        x_i8 = static_cast<int8_t*>(buf);
+        x_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(buf) + qbytes);
+    }
+    int st = sherry_quant_act(x, M, K, x_i8, x_scale, stream);
+    if (st != SHERRY_OK) return st;
+    return sherry_gemm_acc(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
+}
+
+int sherry_linear(const float* x, const void* Wnative, const float* alpha, float* y, int64_t M, int64_t N,
+                  int64_t K, void* stream)
+{
+    if (!y) return SHERRY_ERR_INVALID_ARG;
+    return sherry_linear_ex(x, Wnative, alpha, y, nullptr, nullptr, nullptr, M, N, K, stream);
 }
 
 int sherry_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,

@@ -9,7 +9,11 @@
 // (32 groups = 160 bits = 5 words per row).  Word j of (row r, chunk c) holds
 // canonical stream bytes [20c + 4j, 20c + 4j + 4) of row r, little endian, so
 // group g of the chunk sits at bits [5g, 5g+5) of the 160-bit concatenation
-// of the 5 words.  Memory order: [row tile][chunk][word j][row r in tile].
+// of the 5 words.  Memory order: [row tile][chunk][word j][position p], and
+// plane j is rotated by 8j rows: row r's word j sits at position
+// (r + 8j) mod 128.  A warp reading one word of 32 consecutive rows, and a
+// warp of mma.sync A-fragment lanes reading words c and c+1 of rows g, g+8
+// (lane = 4g + c), both touch 32 distinct shared-memory banks.
 #define SHERRY_TILE_ROWS 128
 #define SHERRY_KCHUNK 128
 #define SHERRY_CHUNK_WORDS 5
@@ -33,6 +37,11 @@ inline bool sherry_shape_ok(int64_t M, int64_t N, int64_t K)
 
 SHERRY_HD inline int64_t sherry_row_tiles(int64_t N) { return (N + SHERRY_TILE_ROWS - 1) / SHERRY_TILE_ROWS; }
 SHERRY_HD inline int64_t sherry_k_chunks(int64_t K) { return (K + SHERRY_KCHUNK - 1) / SHERRY_KCHUNK; }
+// Word index of (word j, row r) inside one (tile, chunk) block.
+SHERRY_HD inline int sherry_word_pos(int j, int r)
+{
+    return j * SHERRY_TILE_ROWS + ((r + 8 * j) & (SHERRY_TILE_ROWS - 1));
+}
 
 // Codes reported through sherry_last_device_status when a bounded wait runs out.
 enum sherry_device_code : unsigned {

@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < SC; ++j)
 #pragma unroll
                     for (int k = 0; k < SHERRY_CHUNK_WORDS; ++k)
-                        w[j][k] = (j < nch) ? codes[(j * SHERRY_CHUNK_WORDS + k) * SHERRY_TILE_ROWS + row] : 0u;
+                        w[j][k] = (j < nch) ? codes[j * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS) + sherry_word_pos(k, row)] : 0u;
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(empty_bar(s));
                 ok = ptx::mbar_wait_bounded(aempty_bar(a), aph ^ 1u, kWaitLimitNs);

@@ -28,17 +28,28 @@ def upload_weights(W: np.ndarray, device="cuda"):
 
 
 def run_gpu(x: np.ndarray, native, alpha_dev, N: int, kernel="auto", with_acc: bool = True):
-    """quant_act + gemm on the device; returns numpy (y, acc, q, s).
+    """quant_act + gemm on the device (kernel "linear": sherry_linear from the
+    fp32 activations); returns numpy (y, acc, q, s).
 
     with_acc=False asks for y only -- the configuration of the benchmark,
     where the tensor-core kernel writes complete output tiles with TMA
     stores -- and returns acc = None."""
     import torch
     xd = torch.from_numpy(np.ascontiguousarray(x)).cuda()
-    q, s = sbm.quant_act(xd)
     M = x.shape[0]
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda") if with_acc else None
-    y = sbm.gemm(q, s, native, alpha_dev, N, acc=acc, kernel=kernel)
+    if kernel == "linear":
+        # fp32 activations straight in (sherry_linear / sherry_linear_ex)
+        if with_acc:
+            q = torch.empty((M, x.shape[1]), dtype=torch.int8, device="cuda")
+            s = torch.empty(M, dtype=torch.float32, device="cuda")
+            y = sbm.linear(xd, native, alpha_dev, N, acc=acc, out_q=q, out_s=s)
+        else:
+            y = sbm.linear(xd, native, alpha_dev, N)
+            q, s = sbm.quant_act(xd)
+    else:
+        q, s = sbm.quant_act(xd)
+        y = sbm.gemm(q, s, native, alpha_dev, N, acc=acc, kernel=kernel)
     torch.cuda.synchronize()
     if acc is None:
         return y.cpu().numpy(), None, q.cpu().numpy(), s.cpu().numpy()

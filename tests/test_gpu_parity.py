@@ -51,6 +51,46 @@ def test_quant_act_ties_and_zero_rows():
     assert np.array_equal(sc.cpu().numpy(), s_o)
 
 
+@pytest.mark.parametrize("path", ["quant_act", "linear"])
+def test_quant_near_rounding_boundaries(path):
+    """Activations within a few ulp of the half-integer rounding boundaries of
+    x / s (where a reciprocal-multiply shortcut could round the other way)
+    and exactly on them: q must equal the oracle's IEEE-division result."""
+    rng = np.random.default_rng(11)
+    K = 4096
+    rows = []
+    for rel in (0.0, 1e-7, 3e-7, 1e-6, 4e-6, 2e-5, 4e-5, 1e-4):
+        a = np.float32(rng.uniform(0.5, 8.0))
+        s = np.float32(a / np.float32(127.0))
+        k = rng.integers(-126, 126, size=K - 1).astype(np.float64)
+        sign = rng.choice([-1.0, 1.0], size=K - 1)
+        x = ((k + 0.5) * (1.0 + sign * rel) * np.float64(s)).astype(np.float32)
+        x = np.clip(x, -a, a)
+        rows.append(np.concatenate([[a], x]).astype(np.float32))
+    x = np.stack(rows)
+    q_o, s_o = oracle.quant_act(x)
+    xd = torch.from_numpy(x).cuda()
+    if path == "quant_act":
+        q, sc = sbm.quant_act(xd)
+    else:
+        N = 256
+        W = synth.weights(0, 9, N, K)
+        native, alpha_d, _, _ = upload_weights(W)
+        for m0 in range(0, x.shape[0], sbm.LINEAR_FUSED_MAX_M):        # fused launches only
+            xs = xd[m0:m0 + sbm.LINEAR_FUSED_MAX_M].contiguous()
+            qq = torch.empty(xs.shape, dtype=torch.int8, device="cuda")
+            ss = torch.empty(xs.shape[0], dtype=torch.float32, device="cuda")
+            acc = torch.empty((xs.shape[0], N), dtype=torch.int32, device="cuda")
+            sbm.linear(xs, native, alpha_d, N, acc=acc, out_q=qq, out_s=ss)
+            torch.cuda.synchronize()
+            assert np.array_equal(qq.cpu().numpy(), q_o[m0:m0 + xs.shape[0]])
+            assert np.array_equal(ss.cpu().numpy().view(np.uint32), s_o[m0:m0 + xs.shape[0]].view(np.uint32))
+        return
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_o)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+
+
 # --------------------------------------------------------------- repack
 @pytest.mark.parametrize("N,K", [(300, 96), (128, 4096), (129, 224), (1, 32)])
 def test_repack_layout(N, K):
@@ -62,7 +102,10 @@ def test_repack_layout(N, K):
     pad = np.zeros((Tn * 128, Kc * 20), dtype=np.uint8)
     pad[:N, :codes.shape[1]] = codes
     expect = pad.reshape(Tn, 128, Kc, 5, 4).view(np.uint32)[..., 0]      # [t][r][c][j]
-    expect = expect.transpose(0, 2, 3, 1).reshape(-1)                   # [t][c][j][r]
+    expect = expect.transpose(0, 2, 3, 1).copy()                        # [t][c][j][r]
+    for j in range(5):                                                  # plane j: row r at (r + 8j) % 128
+        expect[:, :, j, :] = np.roll(expect[:, :, j, :], 8 * j, axis=-1)
+    expect = expect.reshape(-1)
     assert np.array_equal(nat, expect)
 
 
@@ -70,14 +113,23 @@ def test_repack_layout(N, K):
 SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 512),
          (64, 256, 1024), (100, 130, 4096), (129, 257, 160), (256, 512, 2048), (7, 1, 32),
          (2, 4100, 1184), (4, 777, 14336), (1, 640, 9216), (2, 1, 32), (300, 1024, 2048),
-         (200, 388, 4096), (130, 8192, 256)]
+         (200, 388, 4096), (130, 8192, 256), (8, 300, 2048), (16, 129, 4096), (32, 1000, 1024),
+         (9, 77, 16384), (4, 333, 8192), (3, 200, 16384), (5, 50, 160), (24, 2000, 512)]
 
 
-@pytest.mark.parametrize("kernel", ["auto", "tc", "gemv", "simt"])
+def _kernel_serves(kernel: str, M: int, K: int) -> bool:
+    if kernel == "gemv":
+        return M <= sbm.GEMV_MAX_M and K <= 16384
+    if kernel == "decode":
+        return M <= sbm.DECODE_MAX_M
+    return True
+
+
+@pytest.mark.parametrize("kernel", ["auto", "linear", "decode", "tc", "gemv", "simt"])
 @pytest.mark.parametrize("M,N,K", SMALL)
 def test_gemm_small_full(M, N, K, kernel):
-    if kernel == "gemv" and M > sbm.GEMV_MAX_M:
-        pytest.skip("the GEMV kernel serves M <= 4")
+    if not _kernel_serves(kernel, M, K):
+        pytest.skip(f"the {kernel} kernel does not serve M={M}, K={K}")
     W = synth.weights(0, 1, N, K, sigma=0.02)
     x = synth.activations(0, 1, M, K)
     y_o, acc_o, q_o, s_o, codes_o, alpha_o = oracle.reference(x, W)
@@ -87,9 +139,9 @@ def test_gemm_small_full(M, N, K, kernel):
     assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
     assert np.array_equal(acc, acc_o)
     assert_y_close(y, y_o)
-    if kernel in ("auto", "tc"):
+    if kernel in ("auto", "tc", "linear"):
         y2, _, _, _ = run_gpu(x, native, alpha_d, N, kernel, with_acc=False)
-        assert_y_close(y2, y_o)
+        assert np.array_equal(y2, y)
 
 
 def test_gemm_zero_token_and_repeat():
@@ -122,7 +174,7 @@ def _full_size_check(cfg, copy, M_list, K, N, int_mm=True, kernels=("auto",)):
         q_o, s_o = oracle.quant_act(x)
         acc_o = oracle.gemm(q_o, T_rows)
         for kern in kernels:
-            if kern == "gemv" and M > sbm.GEMV_MAX_M:
+            if not _kernel_serves(kern, M, K):
                 continue
             y, acc, q, s = run_gpu(x, native, alpha_d, N, kern)
             assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
@@ -141,12 +193,12 @@ def _full_size_check(cfg, copy, M_list, K, N, int_mm=True, kernels=("auto",)):
 
 @pytest.mark.parametrize("K,N", synth.PROJ_SHAPES)
 def test_config1_decode_full_size(K, N):
-    _full_size_check(1, 0, [1], K, N, kernels=("auto", "tc"))
+    _full_size_check(1, 0, [1], K, N, kernels=("auto", "linear", "tc", "gemv"))
 
 
 @pytest.mark.parametrize("K,N", synth.PROJ_SHAPES)
 def test_config2_small_batch_full_size(K, N):
-    _full_size_check(2, 0, [4, 8, 16, 32], K, N, kernels=("auto", "tc"))
+    _full_size_check(2, 0, [4, 8, 16, 32], K, N, kernels=("auto", "linear", "tc"))
 
 
 @pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096)])
@@ -155,7 +207,7 @@ def test_config3_prefill_full_size(K, N):
 
 
 def test_config4_heavy_tail_full_size():
-    W = _full_size_check(4, 0, [1, 128, 4096], 8192, 28672, kernels=("auto", "tc"))
+    W = _full_size_check(4, 0, [1, 128, 4096], 8192, 28672, kernels=("auto", "linear", "tc"))
     T, _ = oracle.quantise(W)
     assert np.all(np.count_nonzero(T.reshape(28672, -1, 4), axis=2) == 3)
 
@@ -165,7 +217,7 @@ def test_config0_tiny_exact():
     x = synth.config_activations(0, 0, 1, 256)
     y_o, acc_o, *_ = oracle.reference(x, W)
     native, alpha_d, _, _ = upload_weights(W)
-    for kernel in ("auto", "tc", "gemv", "simt"):
+    for kernel in ("auto", "linear", "decode", "tc", "gemv", "simt"):
         y, acc, _, _ = run_gpu(x, native, alpha_d, 128, kernel)
         assert np.array_equal(acc, acc_o)
         assert np.array_equal(y, y_o)
