@@ -13,7 +13,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "libsherry_b200.so")
 SOURCES = ["sherry_cuda.cu", "sherry_host.cpp"]
-HEADERS = ["sherry_internal.h", "ptx.cuh", "tc_gemm.cuh"]
+HEADERS = sorted(f for f in os.listdir(os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc"))
+                 if f.endswith((".h", ".cuh")))
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [

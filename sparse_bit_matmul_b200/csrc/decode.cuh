@@ -54,8 +54,8 @@ struct Params {
     float* y;                    // [M][N] or null
     int32_t* acc;                // [M][N] or null
     int64_t M, N, K, Kc;
-    int G;                       // CTAs; CTA c owns rows [N c / G, N (c+1) / G)
-    int R;                       // largest row count of a CTA
+    int G;                       // CTAs; CTA c owns rows [row_begin(c), row_begin(c+1))
+    int R;                       // largest row count of a CTA, a multiple of 4
     int P;                       // K-parts per row
     int CPT;                     // chunks per K-part
 };
@@ -91,6 +91,13 @@ __device__ __forceinline__ uint32_t expand_code(uint32_t c)
     return word;
 }
 
+// First row of row group g of G: balanced, rounded up to a multiple of 4.
+__host__ __device__ inline int64_t row_begin(int64_t N, int64_t g, int64_t G)
+{
+    const int64_t b = (N * g / G + 3) & ~int64_t(3);
+    return b < N ? b : N;
+}
+
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
@@ -101,6 +108,26 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+
+// N consecutive 32-bit words from a shared address (aligned to 4 N bytes).
+template <int N>
+__device__ __forceinline__ void lds_vec(uint32_t addr, uint32_t (&v)[N]);
+template <>
+__device__ __forceinline__ void lds_vec<1>(uint32_t addr, uint32_t (&v)[1])
+{
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v[0]) : "r"(addr));
+}
+template <>
+__device__ __forceinline__ void lds_vec<2>(uint32_t addr, uint32_t (&v)[2])
+{
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v[0]), "=r"(v[1]) : "r"(addr));
+}
+template <>
+__device__ __forceinline__ void lds_vec<4>(uint32_t addr, uint32_t (&v)[4])
+{
+    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]) : "r"(addr));
+}
+
 template <int MT, bool FUSED>
 __global__ void __launch_bounds__(kMaxThreads, 2)
     sherry_decode_kernel(const Params p)
@@ -109,7 +136,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     const int M = (int)p.M;
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5;
-    const int64_t r0 = p.N * blockIdx.x / p.G, r1 = p.N * (blockIdx.x + 1) / p.G;
+    const int64_t r0 = row_begin(p.N, blockIdx.x, p.G), r1 = row_begin(p.N, blockIdx.x + 1, p.G);
     const int Rc = (int)(r1 - r0);
     const int R = p.R, P = p.P;
     const uint32_t s_base = ptx::smem_u32(smem);
@@ -119,25 +146,34 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     const int QK = (int)p.Kc * SHERRY_KCHUNK;              // bytes per token row of qbuf
 
     // ---- before the wait: this CTA's codes, alpha, the decode table -------------
-    // thread t copies row i = t % R of every (nthr / R)-th chunk: consecutive
-    // lanes read consecutive positions of one word plane
+    // Row groups start at multiples of 4 rows, so 4 consecutive rows of one word
+    // plane are 16 aligned bytes: thread t copies 4-row piece t % R4 of every
+    // (nthr / R4)-th chunk with 16-byte cp.async (4-byte copies for a ragged end);
+    // consecutive lanes read consecutive positions of the plane.
     {
-        const int cstride = nthr / R;
-        const int i = tid % R, c0 = tid / R;
-        if (i < Rc && c0 < cstride) {
-            const int64_t r = r0 + i;
+        const int R4 = (Rc + 3) >> 2;
+        const int cstride = R4 > 0 ? nthr / R4 : 0;
+        const int pi = R4 > 0 ? tid % R4 : 0, cs = R4 > 0 ? tid / R4 : 0;
+        if (cs < cstride) {
+            const int64_t r = r0 + 4 * pi;
             const int rr = (int)(r & 127);
+            const int nr = min(4, Rc - 4 * pi);
             const uint32_t* src = reinterpret_cast<const uint32_t*>(p.wnative) +
                                   (r >> 7) * p.Kc * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS);
             int pos[SHERRY_CHUNK_WORDS];
 #pragma unroll
             for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) pos[j] = sherry_word_pos(j, rr);
-            uint32_t dst = codes_s + 4u * (uint32_t)(c0 * SHERRY_CHUNK_WORDS * R + i);
+            uint32_t dst = codes_s + 4u * (uint32_t)(cs * SHERRY_CHUNK_WORDS * R + 4 * pi);
             const uint32_t dstep = 4u * (uint32_t)(cstride * SHERRY_CHUNK_WORDS * R);
-            for (int c = c0; c < (int)p.Kc; c += cstride) {
+            for (int c = cs; c < (int)p.Kc; c += cstride) {
                 const uint32_t* sc = src + (int64_t)c * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS);
+                if (nr == 4) {
 #pragma unroll
-                for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) cp_async4(dst + 4u * (uint32_t)(j * R), sc + pos[j]);
+                    for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) cp_async16(dst + 4u * (uint32_t)(j * R), sc + pos[j]);
+                } else {
+                    for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
+                        for (int e = 0; e < nr; ++e) cp_async4(dst + 4u * (uint32_t)(j * R + e), sc + pos[j] + e);
+                }
                 dst += dstep;
             }
         }
@@ -229,18 +265,23 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     // instead of queueing in front of this CTA's activation reads
     ptx::pdl_launch_dependents();
 
-    // ---- decode + dp4a -------------------------------------------------------------
+    // ---- decode + dp4a: one row per thread ----------------------------------------
+    // All 32 table loads of a chunk are issued before its dp4a run, which keeps
+    // enough loads in flight with one CTA per SM; the next chunk's code words
+    // are fetched during the current one.
     const int i = tid % R, part = tid / R;
     int32_t acc[MT][4];
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0;
     if (part < P && i < Rc) {
-        const uint32_t* __restrict__ cw = reinterpret_cast<const uint32_t*>(smem + off_codes(M, P, R)) + i;
+        const uint32_t cbase = codes_s + 4u * (uint32_t)i;
+        const uint32_t q_s = s_base + (uint32_t)qoff;
         const int cb = part * p.CPT;
         const int ce = min((int)p.Kc, cb + p.CPT);
         uint32_t wn[SHERRY_CHUNK_WORDS];
 #pragma unroll
-        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) wn[j] = cw[(cb * SHERRY_CHUNK_WORDS + j) * R];
+        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
+            wn[j] = ptx::lds_u32_nv(cbase + 4u * (uint32_t)((cb * SHERRY_CHUNK_WORDS + j) * R));
 #pragma unroll 1
         for (int c = cb; c < ce; ++c) {
             uint32_t w[SHERRY_CHUNK_WORDS + 1];
@@ -249,7 +290,8 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             w[SHERRY_CHUNK_WORDS] = 0;
             if (c + 1 < ce) {
 #pragma unroll
-                for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) wn[j] = cw[((c + 1) * SHERRY_CHUNK_WORDS + j) * R];
+                for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
+                    wn[j] = ptx::lds_u32_nv(cbase + 4u * (uint32_t)(((c + 1) * SHERRY_CHUNK_WORDS + j) * R));
             }
             // table entries of the chunk's 32 codes
             uint32_t e[32];
@@ -264,17 +306,18 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
                 else v = __funnelshift_r(w[wi], w[wi + 1], off - 2);
                 e[g] = ptx::lds_u32_nv((v & 0x7Cu) | table_s);
             }
-            const uint4* __restrict__ qc = reinterpret_cast<const uint4*>(qbuf + c * SHERRY_KCHUNK);
+            const uint32_t qc = q_s + (uint32_t)(c * SHERRY_KCHUNK);
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (m >= M) break;
 #pragma unroll
                 for (int g4 = 0; g4 < 8; ++g4) {
-                    const uint4 qv = qc[(m * QK) / 16 + g4];
-                    acc[m][0] = __dp4a((int)e[4 * g4 + 0], (int)qv.x, acc[m][0]);
-                    acc[m][1] = __dp4a((int)e[4 * g4 + 1], (int)qv.y, acc[m][1]);
-                    acc[m][2] = __dp4a((int)e[4 * g4 + 2], (int)qv.z, acc[m][2]);
-                    acc[m][3] = __dp4a((int)e[4 * g4 + 3], (int)qv.w, acc[m][3]);
+                    uint32_t qv[4];
+                    lds_vec<4>(qc + (uint32_t)(m * QK + 16 * g4), qv);
+                    acc[m][0] = __dp4a((int)e[4 * g4 + 0], (int)qv[0], acc[m][0]);
+                    acc[m][1] = __dp4a((int)e[4 * g4 + 1], (int)qv[1], acc[m][1]);
+                    acc[m][2] = __dp4a((int)e[4 * g4 + 2], (int)qv[2], acc[m][2]);
+                    acc[m][3] = __dp4a((int)e[4 * g4 + 3], (int)qv[3], acc[m][3]);
                 }
             }
         }

@@ -406,14 +406,17 @@ struct DecodePlan {
 
 bool decode_plan(int64_t N, int64_t Kc, int64_t M, int sms, DecodePlan* out)
 {
-    int64_t G = std::min<int64_t>(sms, N);
+    // at least 4 rows per CTA: row boundaries rounded to 4 rows then leave no CTA empty
+    const int64_t gmax = std::max<int64_t>(1, N / 4);
+    int64_t G = std::min<int64_t>(sms, gmax);
     for (int iter = 0; iter < 64; ++iter) {
-        const int64_t R = (N + G - 1) / G;
-        if (R > decode::kMaxThreads) {
-            G = (N + decode::kMaxThreads - 1) / decode::kMaxThreads;
+        const int64_t R = ((N + G - 1) / G + 3 + 3) & ~int64_t(3);     // rounded groups, a multiple of 4
+        const int64_t RQ = R;
+        if (RQ > decode::kMaxThreads) {
+            G = std::min<int64_t>(gmax, (N + decode::kMaxThreads - 1) / decode::kMaxThreads);
             continue;
         }
-        int64_t P = std::max<int64_t>(1, std::min<int64_t>(Kc, decode::kMaxThreads / R));
+        int64_t P = std::max<int64_t>(1, std::min<int64_t>(Kc, decode::kMaxThreads / RQ));
         const int64_t CPT = (Kc + P - 1) / P;
         P = (Kc + CPT - 1) / CPT;
         const int64_t smem = decode::smem_bytes((int)M, (int)P, (int)R, Kc);
@@ -423,12 +426,12 @@ bool decode_plan(int64_t N, int64_t Kc, int64_t M, int sms, DecodePlan* out)
             out->R = (int)R;
             out->P = (int)P;
             out->CPT = (int)CPT;
-            out->threads = (int)((R * P + 31) / 32 * 32);
+            out->threads = (int)std::max<int64_t>(32, (RQ * P + 31) / 32 * 32);
             out->smem = (int)smem;
             return true;
         }
-        if (R == 1) return false;
-        G = (N + R / 2 - 1) / (R / 2);          // halve the rows per CTA
+        if (R <= 4 || G >= gmax) return false;
+        G = std::min<int64_t>(gmax, (N + R / 2 - 1) / (R / 2));       // halve the rows per CTA
     }
     return false;
 }
