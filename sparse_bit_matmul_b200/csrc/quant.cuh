@@ -6,14 +6,16 @@
 // fp32 division), q = clamp(rint(fl(x / s)), -127, 127), round half to even;
 // a == 0 gives s = 0 and q = 0.
 //
-// q is computed without a division for almost every element: with
-// r = fl(1 / s) and t = fl(x * r), |t - x/s| <= |x/s| * (2^-23 + 2^-48) and
-// |fl(x/s) - x/s| <= 2^-24 |x/s|, so |t - fl(x/s)| < 2.3e-5 for
-// |x/s| <= 127.0001.  Unless t lies within kHalfEps = 4e-5 of a half
-// integer, t and fl(x/s) are strictly on the same side of every rounding
-// boundary and rint(t) == rint(fl(x/s)).  Near a boundary (and whenever
-// 1/s is not a finite normal number) the element takes the exact IEEE
-// division.  |rint| never exceeds 127 on the fast path because |x| <= a.
+// q is computed without a division for almost every element: r is the
+// hardware reciprocal approximation of s (rcp.approx, at most 1 ulp off:
+// relative error <= 2^-23) and t = fl(x * r), so |t - x/s| <= |x/s| *
+// (2^-23 + 2^-24 + 2^-47), and |fl(x/s) - x/s| <= 2^-24 |x/s|: together
+// |t - fl(x/s)| < 3.0e-5 for |x/s| <= 127.0001.  Unless t lies within
+// kHalfEps = 4e-5 of a half integer, t and fl(x/s) are strictly on the same
+// side of every rounding boundary and rint(t) == rint(fl(x/s)).  Near a
+// boundary (and whenever s is tiny or r is not finite) the element takes the
+// exact IEEE division, kept out of line.  |rint| never exceeds 127 on the
+// fast path because |x| <= a.
 #pragma once
 
 #include <cstdint>
@@ -30,12 +32,19 @@ struct Scale {
     bool fast;      // the reciprocal path is valid for this token
 };
 
+__device__ __forceinline__ float rcp_approx(float s)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return r;
+}
+
 __device__ __forceinline__ Scale make_scale(float a)
 {
     Scale sc;
     sc.s = __fdiv_rn(a, 127.0f);
     sc.zero = (a == 0.0f);
-    sc.r = __frcp_rn(sc.s);
+    sc.r = rcp_approx(sc.s);
     sc.fast = !sc.zero && sc.s >= 1.0e-30f && isfinite(sc.r) && sc.r < 1.0e30f;
     if (sc.zero) sc.s = 0.0f;
     return sc;
@@ -47,25 +56,32 @@ __device__ __forceinline__ int quantise_exact(float x, float s)
     return r > 127 ? 127 : (r < -127 ? -127 : r);
 }
 
-__device__ __forceinline__ int quantise(float x, const Scale& sc)
+// The exact path for a whole group of four, out of line: rare, and it keeps
+// the division's code and registers away from the common path.
+__device__ __noinline__ uint32_t quantise4_exact(float4 v, float s)
 {
-    if (sc.zero) return 0;
-    if (sc.fast) {
-        const float t = __fmul_rn(x, sc.r);
-        const float rt = rintf(t);
-        if (fabsf(t - rt) < 0.5f - kHalfEps) return (int)rt;
-    }
-    return quantise_exact(x, sc.s);
+    const uint32_t a = (uint32_t)quantise_exact(v.x, s) & 0xFFu;
+    const uint32_t b = (uint32_t)quantise_exact(v.y, s) & 0xFFu;
+    const uint32_t c = (uint32_t)quantise_exact(v.z, s) & 0xFFu;
+    const uint32_t d = (uint32_t)quantise_exact(v.w, s) & 0xFFu;
+    return a | (b << 8) | (c << 16) | (d << 24);
 }
 
 // Four consecutive activations -> four int8 codes packed little endian.
 __device__ __forceinline__ uint32_t quantise4(const float4& v, const Scale& sc)
 {
-    const uint32_t a = (uint32_t)quantise(v.x, sc) & 0xFFu;
-    const uint32_t b = (uint32_t)quantise(v.y, sc) & 0xFFu;
-    const uint32_t c = (uint32_t)quantise(v.z, sc) & 0xFFu;
-    const uint32_t d = (uint32_t)quantise(v.w, sc) & 0xFFu;
-    return a | (b << 8) | (c << 16) | (d << 24);
+    if (sc.zero) return 0u;
+    const float in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed = 0;
+    bool near = !sc.fast;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float t = __fmul_rn(in[e], sc.r);
+        const float rt = rintf(t);
+        near |= !(fabsf(t - rt) < 0.5f - kHalfEps);
+        packed |= ((uint32_t)(int)rt & 0xFFu) << (8 * e);
+    }
+    return near ? quantise4_exact(v, sc.s) : packed;
 }
 
 __device__ __forceinline__ float absmax4(const float4& v)
