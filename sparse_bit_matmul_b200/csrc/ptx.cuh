@@ -227,13 +227,6 @@ __device__ __forceinline__ void red_add_s32(int32_t* p, int32_t v)
     asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ int32_t ld_cg_s32(const int32_t* p)
-{
-    int32_t v;
-    asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 
 // ---- programmatic dependent launch ------------------------------------------
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -295,74 +295,72 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++ds == C::kStages) { ds = 0; dph ^= 1u; }
         }
     } else if (warp == kMmaWarp) {
-        // the whole warp runs the loop (converged); lane 0 issues the MMAs
-        int s = 0, a = 0, d = 0;
-        uint32_t sph = 0, aph = 0, dph = 0;
-        bool issued_any = false, seg_start = true;
-        StageWalk<SC> wk(u0, u1, p.Kc);
-        while (!wk.done()) {
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            bool ok = true;
-            if (seg_start) {
+        // Lane 0 alone issues.  The MMA issue blocks while the tensor pipe is
+        // busy and the pipe holds almost no queued work, so every instruction
+        // this thread runs between two stages is a bubble in the pipe: the
+        // loop keeps one wait pair and a few integer updates per stage, no
+        // warp votes, and segment bookkeeping only at tile ends.
+        if (lane == 0) {
+            int s = 0, a = 0, d = 0;
+            uint32_t sph = 0, aph = 0, dph = 0;
+            bool issued_any = false, ok = true;
+            int64_t u = u0;
+            int64_t seg_end = (u0 / p.Kc + 1) * p.Kc;
+            if (seg_end > u1) seg_end = u1;
+            while (u < u1) {
+                int left = (int)(seg_end - u);     // chunks of this tile segment
                 ok = ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
-                    break;
-                }
-            }
-            ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs) &&
-                 ptx::mbar_wait_bounded(afull_bar(a), aph, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
-                break;
-            }
-            ptx::tc_fence_after();
-            const int nch = wk.nch();
-            if (lane == 0) {
+                if (!ok) break;
                 const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
-                const uint32_t a_tmem = tmem + (uint32_t)(C::kACol0 + a * C::kACols);
-                // descriptor of the stage's first K step; later steps only add
-                // to the start-address field (16-byte units)
-                const uint64_t desc0 = b_desc_sw128(sbase + (uint32_t)s * C::kBStageBytes);
-                const uint32_t acc0 = seg_start ? 0u : 1u;
-                if (nch == SC) {
+                uint32_t acc0 = 0u;
+                while (left > 0) {
+                    ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs) &&
+                         ptx::mbar_wait_bounded(afull_bar(a), aph, kWaitLimitNs);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const uint32_t a_tmem = tmem + (uint32_t)(C::kACol0 + a * C::kACols);
+                    // descriptor of the stage's first K step; later steps only
+                    // add to the start-address field (16-byte units)
+                    const uint64_t desc0 = b_desc_sw128(sbase + (uint32_t)s * C::kBStageBytes);
+                    if (left >= SC) {
 #pragma unroll
-                    for (int j = 0; j < SC; ++j)
+                        for (int j = 0; j < SC; ++j)
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            ptx::mma_i8_ts(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
-                                           desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
-                                           (j == 0 && ks == 0) ? acc0 : 1u);
-                } else {
-                    for (int j = 0; j < nch; ++j)
+                            for (int ks = 0; ks < 4; ++ks)
+                                ptx::mma_i8_ts(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
+                                               desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
+                                               (j == 0 && ks == 0) ? acc0 : 1u);
+                        left -= SC;
+                    } else {
+                        for (int j = 0; j < left; ++j)
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            ptx::mma_i8_ts(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
-                                           desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
-                                           (j == 0 && ks == 0) ? acc0 : 1u);
+                            for (int ks = 0; ks < 4; ++ks)
+                                ptx::mma_i8_ts(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
+                                               desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
+                                               (j == 0 && ks == 0) ? acc0 : 1u);
+                        left = 0;
+                    }
+                    ptx::tc_commit(empty_bar(s));
+                    ptx::tc_commit(aempty_bar(a));
+                    issued_any = true;
+                    acc0 = 1u;
+                    if (++s == C::kStages) { s = 0; sph ^= 1u; }
+                    if (++a == C::kAStages) { a = 0; aph ^= 1u; }
                 }
-                ptx::tc_commit(empty_bar(s));
-                ptx::tc_commit(aempty_bar(a));
-            }
-            __syncwarp();
-            issued_any = true;
-            seg_start = false;
-            if (++s == C::kStages) { s = 0; sph ^= 1u; }
-            if (++a == C::kAStages) { a = 0; aph ^= 1u; }
-            if (wk.next()) {
-                if (lane == 0) ptx::tc_commit(dfull_bar(d));
-                __syncwarp();
+                if (!ok) break;
+                ptx::tc_commit(dfull_bar(d));
                 if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
-                seg_start = true;
+                u = seg_end;
+                seg_end += p.Kc;
+                if (seg_end > u1) seg_end = u1;
             }
-        }
-        if (issued_any) {
-            // all MMAs of this warp complete before tensor memory is freed
-            if (lane == 0) ptx::tc_commit(drain_bar);
-            __syncwarp();
-            const bool ok = ptx::mbar_wait_bounded(drain_bar, 0, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok) && lane == 0)
-                atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
+            if (!ok) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
+            if (issued_any) {
+                // all MMAs of this thread complete before tensor memory is freed
+                ptx::tc_commit(drain_bar);
+                if (!ptx::mbar_wait_bounded(drain_bar, 0, kWaitLimitNs))
+                    atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
+            }
         }
     } else if (warp >= kDecWarp0 && warp < kDecWarp0 + 4 * kDecGroups) {
         const int grp = (warp - kDecWarp0) / 4;
@@ -532,15 +530,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::named_bar_sync(1, 128);
                 if (*last_flag) {
                     __threadfence();
-                    for (int j = 0; j < BN; ++j) {
-                        const int64_t m = cur_tm * BN + j;
-                        if (m >= p.M) break;
-                        int32_t* cell = wsl + j * SHERRY_TILE_ROWS + r;
-                        const int32_t a32 = ptx::ld_cg_s32(cell);
-                        *cell = 0;
-                        if (n < p.N) {
-                            if (p.acc) p.acc[m * p.N + n] = a32;
-                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, al), sc_s[j]);
+                    // 16 independent L2 loads in flight per batch: one round
+                    // trip per 16 tokens, not one per token
+                    const int64_t mleft = p.M - cur_tm * BN;
+                    const int jn = mleft < BN ? (int)mleft : BN;
+                    for (int j0 = 0; j0 < jn; j0 += 16) {
+                        int32_t v[16];
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            v[jj] = (j0 + jj < jn) ? __ldcg(wsl + (j0 + jj) * SHERRY_TILE_ROWS + r) : 0;
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) {
+                            const int j = j0 + jj;
+                            if (j >= jn) break;
+                            const int64_t m = cur_tm * BN + j;
+                            wsl[j * SHERRY_TILE_ROWS + r] = 0;
+                            if (n < p.N) {
+                                if (p.acc) p.acc[m * p.N + n] = v[jj];
+                                if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)v[jj], al), sc_s[j]);
+                            }
                         }
                     }
                     if (etid == 0) atomicExch(p.counters + slot, 0u);
