@@ -295,72 +295,86 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++ds == C::kStages) { ds = 0; dph ^= 1u; }
         }
     } else if (warp == kMmaWarp) {
-        // Lane 0 alone issues.  The MMA issue blocks while the tensor pipe is
-        // busy and the pipe holds almost no queued work, so every instruction
-        // this thread runs between two stages is a bubble in the pipe: the
-        // loop keeps one wait pair and a few integer updates per stage, no
-        // warp votes, and segment bookkeeping only at tile ends.
-        if (lane == 0) {
-            int s = 0, a = 0, d = 0;
-            uint32_t sph = 0, aph = 0, dph = 0;
-            bool issued_any = false, ok = true;
-            int64_t u = u0;
-            int64_t seg_end = (u0 / p.Kc + 1) * p.Kc;
-            if (seg_end > u1) seg_end = u1;
-            while (u < u1) {
-                int left = (int)(seg_end - u);     // chunks of this tile segment
-                ok = ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs);
-                if (!ok) break;
-                const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
-                uint32_t acc0 = 0u;
-                while (left > 0) {
+        // The MMA issue blocks while the tensor pipe is busy and the pipe holds
+        // almost no queued work, so every instruction between two MMAs is a
+        // bubble.  Hence: the whole warp runs the loop converged, with every
+        // loop value warp-uniform (votes make the wait results uniform), and
+        // one elected lane issues inside the MMA's own instruction sequence;
+        // and the next stage's barriers are tested (non-blocking) before the
+        // current stage's MMAs, so a stage whose inputs are ready starts with
+        // no wait.
+        int s = 0, a = 0, d = 0;
+        uint32_t sph = 0, aph = 0, dph = 0;
+        bool issued_any = false, ok = true;
+        bool ready = false;                      // this stage's full and afull already seen complete
+        int64_t u = u0;
+        int64_t seg_end = (u0 / p.Kc + 1) * p.Kc;
+        if (seg_end > u1) seg_end = u1;
+        while (u < u1) {
+            int left = (int)(seg_end - u);         // chunks of this tile segment
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs));
+            if (!ok) break;
+            const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
+            uint32_t acc0 = 0u;
+            while (left > 0) {
+                if (!ready) {
                     ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs) &&
                          ptx::mbar_wait_bounded(afull_bar(a), aph, kWaitLimitNs);
+                    ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
-                    ptx::tc_fence_after();
-                    const uint32_t a_tmem = tmem + (uint32_t)(C::kACol0 + a * C::kACols);
-                    // descriptor of the stage's first K step; later steps only
-                    // add to the start-address field (16-byte units)
-                    const uint64_t desc0 = b_desc_sw128(sbase + (uint32_t)s * C::kBStageBytes);
-                    if (left >= SC) {
-#pragma unroll
-                        for (int j = 0; j < SC; ++j)
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                ptx::mma_i8_ts(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
-                                               desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
-                                               (j == 0 && ks == 0) ? acc0 : 1u);
-                        left -= SC;
-                    } else {
-                        for (int j = 0; j < left; ++j)
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                ptx::mma_i8_ts(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
-                                               desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
-                                               (j == 0 && ks == 0) ? acc0 : 1u);
-                        left = 0;
-                    }
-                    ptx::tc_commit(empty_bar(s));
-                    ptx::tc_commit(aempty_bar(a));
-                    issued_any = true;
-                    acc0 = 1u;
-                    if (++s == C::kStages) { s = 0; sph ^= 1u; }
-                    if (++a == C::kAStages) { a = 0; aph ^= 1u; }
                 }
-                if (!ok) break;
-                ptx::tc_commit(dfull_bar(d));
-                if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
-                u = seg_end;
-                seg_end += p.Kc;
-                if (seg_end > u1) seg_end = u1;
+                ptx::tc_fence_after();
+                const int s1 = (s + 1 == C::kStages) ? 0 : s + 1;
+                const int a1 = (a + 1 == C::kAStages) ? 0 : a + 1;
+                const uint32_t sph1 = (s + 1 == C::kStages) ? sph ^ 1u : sph;
+                const uint32_t aph1 = (a + 1 == C::kAStages) ? aph ^ 1u : aph;
+                // both tests issue before the MMAs; their results are read
+                // only after the stage's last MMA
+                const uint32_t t_full = ptx::mbar_test(full_bar(s1), sph1);
+                const uint32_t t_a = ptx::mbar_test(afull_bar(a1), aph1);
+                const uint32_t a_tmem = tmem + (uint32_t)(C::kACol0 + a * C::kACols);
+                // descriptor of the stage's first K step; later steps only
+                // add to the start-address field (16-byte units)
+                const uint64_t desc0 = b_desc_sw128(sbase + (uint32_t)s * C::kBStageBytes);
+                if (left >= SC) {
+#pragma unroll
+                    for (int j = 0; j < SC; ++j)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            ptx::mma_i8_ts_elect(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
+                                                 desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
+                                                 (j == 0 && ks == 0) ? acc0 : 1u);
+                    left -= SC;
+                } else {
+                    for (int j = 0; j < left; ++j)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            ptx::mma_i8_ts_elect(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
+                                                 desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
+                                                 (j == 0 && ks == 0) ? acc0 : 1u);
+                    left = 0;
+                }
+                ptx::tc_commit_elect(empty_bar(s));
+                ptx::tc_commit_elect(aempty_bar(a));
+                issued_any = true;
+                acc0 = 1u;
+                s = s1; a = a1; sph = sph1; aph = aph1;
+                ready = __all_sync(0xffffffffu, (t_full & t_a) != 0u);
             }
-            if (!ok) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
-            if (issued_any) {
-                // all MMAs of this thread complete before tensor memory is freed
-                ptx::tc_commit(drain_bar);
-                if (!ptx::mbar_wait_bounded(drain_bar, 0, kWaitLimitNs))
-                    atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
-            }
+            if (!ok) break;
+            ptx::tc_commit_elect(dfull_bar(d));
+            if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
+            u = seg_end;
+            seg_end += p.Kc;
+            if (seg_end > u1) seg_end = u1;
+        }
+        if (!ok && lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
+        if (issued_any) {
+            // all MMAs of this warp complete before tensor memory is freed
+            ptx::tc_commit_elect(drain_bar);
+            const bool done = ptx::mbar_wait_bounded(drain_bar, 0, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, done) && lane == 0)
+                atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
         }
     } else if (warp >= kDecWarp0 && warp < kDecWarp0 + 4 * kDecGroups) {
         const int grp = (warp - kDecWarp0) / 4;
@@ -376,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nch = wk.nch();
             const bool mine = turn == grp;
             if (mine) {
-                if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                // no per-stage abort poll: after another role gave up, this
+                // wait runs out by itself and the group leaves
                 bool ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
