@@ -245,50 +245,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_holder;
 
     if (warp == kProducerWarp) {
-        // the whole warp runs the loop (converged); lane 0 issues the copies
-        int64_t issued = 0;
-        int64_t tm = 0, tn = 0;
-        {
-            const int64_t tile = u0 / p.Kc;
-            tm = tile / p.TN;
-            tn = tile - tm * p.TN;
-        }
+        // Converged warp, elected-lane issue and a non-blocking test of the
+        // next slot, for the same reason as the MMA loop below: a copy issued
+        // late delays every role after it.
         int s = 0;
         uint32_t ph = 0;
-        StageWalk<SC> wk(u0, u1, p.Kc);
-        while (!wk.done()) {
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            const bool ok = ptx::mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_PRODUCER);
-                break;
+        bool ready = false;                      // empty(s) already seen complete
+        bool ok = true;
+        int64_t issued = 0;
+        int64_t tile = u0 / p.Kc;
+        int64_t tm = tile / p.TN, tn = tile - tm * p.TN;
+        int64_t u = u0;
+        int64_t seg_end = (tile + 1) * p.Kc < u1 ? (tile + 1) * p.Kc : u1;
+        while (u < u1) {
+            int c = (int)(u - tile * p.Kc);        // K chunk within the tile
+            const uint8_t* src = p.wnative + (tn * p.Kc + c) * (int64_t)kChunkCodeBytes;
+            const int32_t ty = (int32_t)(tm * BN);
+            int left = (int)(seg_end - u);
+            while (left > 0) {
+                const int nch = left < SC ? left : SC;
+                if (!ready) {
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs));
+                    if (!ok) break;
+                }
+                const int s1 = (s + 1 == C::kStages) ? 0 : s + 1;
+                const uint32_t ph1 = (s + 1 == C::kStages) ? ph ^ 1u : ph;
+                const uint32_t t_e = ptx::mbar_test(empty_bar(s1), ph1 ^ 1u);
+                ptx::mbar_arrive_expect_tx_elect(full_bar(s), (uint32_t)(nch * (kChunkCodeBytes + C::kBChunkBytes)));
+                ptx::bulk_g2s_elect(sbase + C::kOffCodes + (uint32_t)s * C::kCodeStageBytes, src,
+                                    (uint32_t)(nch * kChunkCodeBytes), full_bar(s));
+                if (nch == SC) {
+#pragma unroll
+                    for (int j = 0; j < SC; ++j)
+                        ptx::tma_load_2d_elect(sbase + (uint32_t)(s * C::kBStageBytes + j * C::kBChunkBytes), &xmap,
+                                               (c + j) * SHERRY_KCHUNK, ty, full_bar(s));
+                } else {
+                    for (int j = 0; j < nch; ++j)
+                        ptx::tma_load_2d_elect(sbase + (uint32_t)(s * C::kBStageBytes + j * C::kBChunkBytes), &xmap,
+                                               (c + j) * SHERRY_KCHUNK, ty, full_bar(s));
+                }
+                src += nch * kChunkCodeBytes;
+                c += nch;
+                left -= nch;
+                ++issued;
+                s = s1;
+                ph = ph1;
+                ready = __all_sync(0xffffffffu, t_e != 0u);
             }
-            const int nch = wk.nch();
-            const int64_t c = wk.chunk();
-            if (lane == 0) {
-                ptx::mbar_arrive_expect_tx(full_bar(s), (uint32_t)(nch * (kChunkCodeBytes + C::kBChunkBytes)));
-                ptx::bulk_g2s(sbase + C::kOffCodes + (uint32_t)s * C::kCodeStageBytes,
-                              p.wnative + (tn * p.Kc + c) * (int64_t)kChunkCodeBytes,
-                              (uint32_t)(nch * kChunkCodeBytes), full_bar(s));
-                for (int j = 0; j < nch; ++j)
-                    ptx::tma_load_2d(sbase + (uint32_t)(s * C::kBStageBytes + j * C::kBChunkBytes), &xmap,
-                                     (int32_t)((c + j) * SHERRY_KCHUNK), (int32_t)(tm * BN), full_bar(s));
-            }
-            __syncwarp();
-            ++issued;
-            if (++s == C::kStages) { s = 0; ph ^= 1u; }
-            if (wk.next()) {
-                if (++tn == p.TN) { tn = 0; ++tm; }
-            }
+            if (!ok) break;
+            u = seg_end;
+            ++tile;
+            if (++tn == p.TN) { tn = 0; ++tm; }
+            seg_end = seg_end + p.Kc < u1 ? seg_end + p.Kc : u1;
         }
+        if (!ok && lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_PRODUCER);
         // every copy issued has landed before the CTA may exit (in the
         // normal flow the consumers already waited for all of them)
         const int64_t from = issued > C::kStages ? issued - C::kStages : 0;
         int ds = (int)(from % C::kStages);
         uint32_t dph = (uint32_t)((from / C::kStages) & 1);
         for (int64_t i = from; i < issued; ++i) {
-            const bool ok = ptx::mbar_wait_bounded(full_bar(ds), dph, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) {
+            const bool landed = ptx::mbar_wait_bounded(full_bar(ds), dph, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, landed)) {
                 if (lane == 0) atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
                 break;
             }
