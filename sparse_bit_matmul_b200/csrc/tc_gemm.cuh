@@ -19,12 +19,14 @@
 //     descriptor; rows past M and columns past K are zero-filled by TMA.
 //   * D (int32 accumulators) lives in tensor memory; epilogue warps read it
 //     with tcgen05.ld and apply the two fp32 products.
-// Work is split "stream-K": the (token tile, row tile, K chunk) units are
-// cut into one contiguous range per CTA (one CTA per SM), so every SM gets
-// the same number of K chunks whatever the shape.  A tile whose K range spans
+// Work is split so that every SM gets the same number of K chunks whatever
+// the shape (one CTA per SM): each CTA first takes an even share of the
+// units (token tile, row tile, K chunk) of the T mod G tiles left over, then
+// T div G whole tiles of its own (SegWalk).  A tile whose K range spans
 // several CTAs is summed exactly with int32 red.add into a workspace slot;
 // the last contributor (an atomic counter) runs the epilogue and clears the
-// slot and counter, so the workspace is all zero between calls.
+// slot and counter, so the workspace is all zero between calls.  The split
+// tiles come first, so their reductions overlap the whole tiles after them.
 //
 // A pipeline stage carries SC consecutive K chunks of one tile (one bulk copy
 // of SC * 2560 bytes of codes, SC 2D TMA boxes of activations, SC * 4 MMAs),
@@ -113,11 +115,90 @@ struct Params {
     int y_tma;                  // y rows 16-byte multiples: complete tiles leave through TMA stores
 };
 
-// CTA that owns unit u when U units are cut into G contiguous ranges
-// [floor(U b / G), floor(U (b+1) / G)).
-__device__ __forceinline__ int64_t owner_of(int64_t u, int64_t U, int64_t G)
+// The work of one CTA as a sequence of tile segments (a segment = chunks
+// [cb, ce) of one tile; units are numbered tile-major, unit = tile * Kc +
+// chunk).  With T tiles and G CTAs, the last R = T mod G tiles are split
+// stream-K: their RU = R * Kc units are cut into G contiguous shares (each
+// under one tile; when RU < G, one unit to each of the first RU CTAs, so
+// that no share is empty), walked first.  Then every CTA walks F = T div G whole tiles of
+// its own.  So every CTA gets the same number of units within one, the
+// tiles summed across CTAs come first (their reductions overlap the later
+// tiles), and every CTA ends on whole tiles.  All roles walk this sequence.
+struct SegWalk {
+    int64_t Kc, tile, cb, ce, end_u, r1_tile, r1_end_tile;
+    int range;                                  // 0 split share, 1 own tiles, 2 done
+    __device__ SegWalk(const Params& p, int64_t b, int64_t G)
+    {
+        Kc = p.Kc;
+        const int64_t T = p.TM * p.TN;
+        const int64_t F = T / G, R = T - F * G;
+        const int64_t L0 = (T - R) * Kc, RU = R * Kc;
+        r1_tile = b * F;
+        r1_end_tile = (b + 1) * F;
+        int64_t a0, a1;
+        if (RU >= G) {
+            a0 = L0 + RU * b / G;
+            a1 = L0 + RU * (b + 1) / G;
+        } else {
+            a0 = L0 + b;
+            a1 = a0 + (b < RU ? 1 : 0);
+        }
+        if (a0 < a1) {
+            range = 0;
+            end_u = a1;
+            tile = a0 / Kc;
+            cb = a0 - tile * Kc;
+            const int64_t te = (tile + 1) * Kc;
+            ce = (te < a1 ? te : a1) - tile * Kc;
+        } else {
+            start_own();
+        }
+    }
+    __device__ void start_own()
+    {
+        if (r1_tile < r1_end_tile) {
+            range = 1;
+            tile = r1_tile;
+            cb = 0;
+            ce = Kc;
+        } else {
+            range = 2;
+        }
+    }
+    __device__ bool done() const { return range == 2; }
+    __device__ bool complete() const { return cb == 0 && ce == Kc; }
+    __device__ void next()
+    {
+        if (range == 0) {
+            const int64_t u = tile * Kc + ce;
+            if (u < end_u) {
+                ++tile;
+                cb = 0;
+                ce = (end_u - u) < Kc ? (end_u - u) : Kc;
+            } else {
+                start_own();
+            }
+        } else if (++tile >= r1_end_tile) {
+            range = 2;
+        }
+    }
+};
+
+// First and last CTA of a split tile t (one of the last R tiles): the owners
+// of its first and last unit among the G shares of the split units.
+__device__ __forceinline__ void split_owners(const Params& p, int64_t t, int64_t G, int64_t* bf, int64_t* bl)
 {
-    return ((u + 1) * G - 1) / U;
+    const int64_t T = p.TM * p.TN;
+    const int64_t R = T - (T / G) * G;
+    const int64_t RU = R * p.Kc;
+    const int64_t u = (t - (T - R)) * p.Kc;
+    if (RU >= G) {
+        *bf = ((u + 1) * G - 1) / RU;
+        *bl = ((u + p.Kc) * G - 1) / RU;
+    } else {
+        *bf = u;
+        *bl = u + p.Kc - 1;
+    }
 }
 
 __device__ __forceinline__ uint64_t b_desc_sw128(uint32_t smem_addr)
@@ -196,10 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // this CTA's unit range
     const int64_t G = gridDim.x;
-    const int64_t u0 = (p.U * (int64_t)blockIdx.x) / G;
-    const int64_t u1 = (p.U * ((int64_t)blockIdx.x + 1)) / G;
 
     if (threadIdx.x < 32) {
         // code -> four int8 weights of the group, byte i = position i
@@ -253,15 +331,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ready = false;                      // empty(s) already seen complete
         bool ok = true;
         int64_t issued = 0;
-        int64_t tile = u0 / p.Kc;
-        int64_t tm = tile / p.TN, tn = tile - tm * p.TN;
-        int64_t u = u0;
-        int64_t seg_end = (tile + 1) * p.Kc < u1 ? (tile + 1) * p.Kc : u1;
-        while (u < u1) {
-            int c = (int)(u - tile * p.Kc);        // K chunk within the tile
+        SegWalk w(p, blockIdx.x, G);
+        while (!w.done()) {
+            const int64_t tm = w.tile / p.TN, tn = w.tile - tm * p.TN;
+            int c = (int)w.cb;                     // K chunk within the tile
             const uint8_t* src = p.wnative + (tn * p.Kc + c) * (int64_t)kChunkCodeBytes;
             const int32_t ty = (int32_t)(tm * BN);
-            int left = (int)(seg_end - u);
+            int left = (int)(w.ce - w.cb);
             while (left > 0) {
                 const int nch = left < SC ? left : SC;
                 if (!ready) {
@@ -293,10 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ready = __all_sync(0xffffffffu, t_e != 0u);
             }
             if (!ok) break;
-            u = seg_end;
-            ++tile;
-            if (++tn == p.TN) { tn = 0; ++tm; }
-            seg_end = seg_end + p.Kc < u1 ? seg_end + p.Kc : u1;
+            w.next();
         }
         if (!ok && lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_PRODUCER);
         // every copy issued has landed before the CTA may exit (in the
@@ -325,11 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sph = 0, aph = 0, dph = 0;
         bool issued_any = false, ok = true;
         bool ready = false;                      // this stage's full and afull already seen complete
-        int64_t u = u0;
-        int64_t seg_end = (u0 / p.Kc + 1) * p.Kc;
-        if (seg_end > u1) seg_end = u1;
-        while (u < u1) {
-            int left = (int)(seg_end - u);         // chunks of this tile segment
+        SegWalk w(p, blockIdx.x, G);
+        while (!w.done()) {
+            int left = (int)(w.ce - w.cb);         // chunks of this tile segment
             ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(dempty_bar(d), dph ^ 1u, kWaitLimitNs));
             if (!ok) break;
             const uint32_t d_tmem = tmem + (uint32_t)(d * BN);
@@ -382,9 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             ptx::tc_commit_elect(dfull_bar(d));
             if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
-            u = seg_end;
-            seg_end += p.Kc;
-            if (seg_end > u1) seg_end = u1;
+            w.next();
         }
         if (!ok && lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_MMA);
         if (issued_any) {
@@ -403,9 +472,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int s = 0, a = 0;
         uint32_t sph = 0, aph = 0;
         int turn = 0;                               // iteration index modulo kDecGroups
-        StageWalk<SC> wk(u0, u1, p.Kc);
-        for (; !wk.done(); wk.next(), turn = (turn + 1 == kDecGroups) ? 0 : turn + 1) {
-            const int nch = wk.nch();
+        bool quit = false;
+        SegWalk w(p, blockIdx.x, G);
+        for (; !w.done() && !quit; w.next()) {
+          for (int left = (int)(w.ce - w.cb); left > 0; left -= SC, turn = (turn + 1 == kDecGroups) ? 0 : turn + 1) {
+            const int nch = left < SC ? left : SC;
             const bool mine = turn == grp;
             if (mine) {
                 // no per-stage abort poll: after another role gave up, this
@@ -413,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
+                    quit = true;
                     break;
                 }
                 const uint32_t* codes =
@@ -428,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = ptx::mbar_wait_bounded(aempty_bar(a), aph ^ 1u, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
+                    quit = true;
                     break;
                 }
                 ptx::tc_fence_after();
@@ -455,6 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (++s == C::kStages) { s = 0; sph ^= 1u; }
             if (++a == C::kAStages) { a = 0; aph ^= 1u; }
+          }
         }
     } else if (warp >= kEpiWarp0) {
         const int quad = warp & 3;
@@ -462,19 +536,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         const int etid = threadIdx.x - kEpiWarp0 * 32;     // 0..127
         int64_t seg = 0;
-        int64_t u = u0;
-        int64_t tile = u0 / p.Kc;
-        int64_t tm = tile / p.TN, tn = tile - (tile / p.TN) * p.TN;
         int d = 0;
         uint32_t dph = 0;
         uint32_t stage_slice = 0;                  // output slices staged so far
-        while (u < u1) {
-            const int64_t cb = u - tile * p.Kc;
-            const int64_t seg_end = (tile + 1) * p.Kc < u1 ? (tile + 1) * p.Kc : u1;
-            const int64_t ce = seg_end - tile * p.Kc;
-            u = seg_end;
+        SegWalk w(p, blockIdx.x, G);
+        for (; !w.done(); w.next()) {
+            const int64_t tile = w.tile;
+            const int64_t tm = tile / p.TN, tn = tile - tm * p.TN;
             const int64_t n = tn * SHERRY_TILE_ROWS + r;
-            const bool complete = (cb == 0 && ce == p.Kc);
+            const bool complete = w.complete();
             // the tile's token scales and this row's alpha do not depend on
             // the MMAs: fetch them into shared memory (double-buffered by
             // segment) before waiting for the accumulators
@@ -495,8 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             int64_t slot = 0, nparts = 1;
             if (!complete) {
-                const int64_t bf = owner_of(tile * p.Kc, p.U, G);
-                const int64_t bl = owner_of(tile * p.Kc + p.Kc - 1, p.U, G);
+                int64_t bf = 0, bl = 0;
+                split_owners(p, tile, G, &bf, &bl);
                 slot = bf;
                 nparts = bl - bf + 1;
             }
@@ -550,8 +620,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++seg;
             if (++d == C::kDBufs) { d = 0; dph ^= 1u; }
             const int64_t cur_tm = tm;
-            ++tile;
-            if (++tn == p.TN) { tn = 0; ++tm; }
             if (!complete) {
                 __threadfence();
                 ptx::named_bar_sync(1, 128);

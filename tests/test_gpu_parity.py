@@ -114,7 +114,12 @@ SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 5
          (64, 256, 1024), (100, 130, 4096), (129, 257, 160), (256, 512, 2048), (7, 1, 32),
          (2, 4100, 1184), (4, 777, 14336), (1, 640, 9216), (2, 1, 32), (300, 1024, 2048),
          (200, 388, 4096), (130, 8192, 256), (8, 300, 2048), (16, 129, 4096), (32, 1000, 1024),
-         (9, 77, 16384), (4, 333, 8192), (3, 200, 16384), (5, 50, 160), (24, 2000, 512)]
+         (9, 77, 16384), (4, 333, 8192), (3, 200, 16384), (5, 50, 160), (24, 2000, 512),
+         # whole tiles per CTA plus split tiles on a 148-SM grid: 149 tiles
+         # of one chunk (one split unit), 150 tiles of five chunks (split
+         # units fewer than CTAs), 200 tiles of eight chunks (split units
+         # shared out by floor division)
+         (100, 19072, 128), (300, 6400, 640), (520, 5120, 1024)]
 
 
 def _kernel_serves(kernel: str, M: int, K: int) -> bool:
