@@ -237,15 +237,16 @@ int get_workspace(size_t bytes, cudaStream_t stream, void** out)
     return SHERRY_OK;
 }
 
-// fp32 y [M][N]: boxes of 128 rows n x 16 tokens m (no swizzle); needs rows
-// of whole 16-byte units (N % 4 == 0) and a 16-byte aligned base.
-int make_y_map(CUtensorMap* map, const float* y, int64_t M, int64_t N)
+// fp32 y [M][N]: boxes of 32 rows n x box_m tokens m (no swizzle), one per
+// epilogue warp; needs rows of whole 16-byte units (N % 4 == 0) and a
+// 16-byte aligned base.
+int make_y_map(CUtensorMap* map, const float* y, int64_t M, int64_t N, int box_m)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return SHERRY_ERR_CUDA;
     cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
     cuuint64_t strides[1] = {(cuuint64_t)N * 4};
-    cuuint32_t box[2] = {SHERRY_TILE_ROWS, 16};
+    cuuint32_t box[2] = {32, (cuuint32_t)box_m};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(y), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -310,7 +311,7 @@ int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alp
     if (st != SHERRY_OK) return st;
     std::memset(&ymap, 0, sizeof(ymap));
     p.y_tma = (y && N % 4 == 0 && aligned16(y)) ? 1 : 0;
-    if (p.y_tma && make_y_map(&ymap, y, M, N) != SHERRY_OK) p.y_tma = 0;
+    if (p.y_tma && make_y_map(&ymap, y, M, N, C::kSlice) != SHERRY_OK) p.y_tma = 0;
 
     // at least half of the SM's shared memory so that exactly one CTA (and
     // one 512-column tensor-memory allocation) lives on each SM
@@ -578,7 +579,7 @@ int launch_tc_noalloc(const int8_t* x, const float* xs, const void* wn, const fl
     if (st != SHERRY_OK) return st;
     std::memset(&ymap, 0, sizeof(ymap));
     p.y_tma = (y && N % 4 == 0 && aligned16(y)) ? 1 : 0;
-    if (p.y_tma && make_y_map(&ymap, y, M, N) != SHERRY_OK) p.y_tma = 0;
+    if (p.y_tma && make_y_map(&ymap, y, M, N, C::kSlice) != SHERRY_OK) p.y_tma = 0;
     const int smem = std::max(C::kSmemBytes, 120 * 1024);
     if (smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
     if (cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN, SC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=

@@ -90,9 +90,11 @@ struct Cfg {
     static constexpr int kNumBars = 2 * kStages + 2 * kAStages + 2 * kDBufs + 1;
     static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
     static constexpr int kMiscBytes = 64 + 2 * BN * 4;   // tmem holder, flags, token scales [2][BN]
-    // output staging for TMA stores: two slices of [16 tokens][128 rows] fp32
+    // output staging for TMA stores: per epilogue warp two slices of
+    // [kSlice tokens][32 rows] fp32
+    static constexpr int kSlice = BN < 32 ? BN : 32;
     static constexpr int kOffStaging = (kOffMisc + kMiscBytes + 127) & ~127;
-    static constexpr int kStagingBytes = 2 * 16 * 128 * 4;
+    static constexpr int kStagingBytes = 4 * 2 * kSlice * 32 * 4;
     static constexpr int kSmemBytes = kOffStaging + kStagingBytes + 1024;   // + alignment slack
     // instruction descriptor: s32 accumulate, signed int8 A and B, both
     // K-major, N = BN, M = 128
@@ -572,33 +574,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int32_t* wsl = p.ws + slot * (int64_t)BN * SHERRY_TILE_ROWS;
             const bool via_tma = complete && p.y_tma && p.y && !p.acc;
+            if (via_tma) {
+                // Each warp stores its own 32 rows x kSlice tokens through TMA
+                // from its own double-buffered staging, with its own bulk
+                // groups: no barrier across the epilogue warps per slice.
+                constexpr int SL = C::kSlice;
+                float* stg_w = reinterpret_cast<float*>(smem + C::kOffStaging) + quad * (2 * SL * 32);
 #pragma unroll 1
-            for (int j0 = 0; j0 < BN; j0 += 16) {
-                if (via_tma && tm * BN + j0 >= p.M) break;     // rows past M: nothing to store
-                uint32_t v[16];
-                if (via_tma) {
-                    // staging buffer of this slice is free once the store
-                    // issued two slices ago has read it
-                    if (etid == 0) ptx::bulk_wait_group_read<1>();
-                    ptx::named_bar_sync(1, 128);
-                }
-                ptx::tmem_ld_32x32b_x16(lane_base + (uint32_t)(d * BN + j0), v);
-                ptx::tmem_wait_ld();
-                if (via_tma) {
-                    float* stg = reinterpret_cast<float*>(smem + C::kOffStaging) + (stage_slice & 1) * (16 * 128);
+                for (int j0 = 0; j0 < BN; j0 += SL) {
+                    if (tm * BN + j0 >= p.M) break;     // tokens past M: nothing to store
+                    uint32_t v[SL];
+                    if constexpr (SL == 32) ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(d * BN + j0), v);
+                    else ptx::tmem_ld_32x32b_x16(lane_base + (uint32_t)(d * BN + j0), v);
+                    // this slice's buffer is free once the store issued two
+                    // slices ago has read it
+                    if (lane == 0) ptx::bulk_wait_group_read<1>();
+                    __syncwarp();
+                    ptx::tmem_wait_ld();
+                    float* stg = stg_w + (stage_slice & 1) * (SL * 32);
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        stg[jj * 128 + r] = __fmul_rn(__fmul_rn((float)(int32_t)v[jj], al), sc_s[j0 + jj]);
+                    for (int jj = 0; jj < SL; ++jj)
+                        stg[jj * 32 + lane] = __fmul_rn(__fmul_rn((float)(int32_t)v[jj], al), sc_s[j0 + jj]);
                     ptx::fence_proxy_async_smem();
-                    ptx::named_bar_sync(1, 128);
-                    if (etid == 0) {
-                        ptx::tma_store_2d(&ymap, (int32_t)(tn * SHERRY_TILE_ROWS), (int32_t)(tm * BN + j0),
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::tma_store_2d(&ymap, (int32_t)(tn * SHERRY_TILE_ROWS + quad * 32), (int32_t)(tm * BN + j0),
                                           ptx::smem_u32(stg));
                         ptx::bulk_commit_group();
                     }
                     ++stage_slice;
-                    continue;
                 }
+            }
+#pragma unroll 1
+            for (int j0 = 0; j0 < (via_tma ? 0 : BN); j0 += 16) {
+                uint32_t v[16];
+                ptx::tmem_ld_32x32b_x16(lane_base + (uint32_t)(d * BN + j0), v);
+                ptx::tmem_wait_ld();
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     const int64_t m = tm * BN + j0 + jj;
@@ -659,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // shared memory stays valid until every TMA store has read it
-        if (etid == 0) ptx::bulk_wait_group<0>();
+        if (lane == 0) ptx::bulk_wait_group<0>();
     }
 
     __syncwarp();
