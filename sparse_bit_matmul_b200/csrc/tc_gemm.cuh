@@ -129,7 +129,7 @@ struct Params {
 struct SegWalk {
     int64_t Kc, tile, cb, ce, end_u, r1_tile, r1_end_tile;
     int range;                                  // 0 split share, 1 own tiles, 2 done
-    __device__ SegWalk(const Params& p, int64_t b, int64_t G)
+    SHERRY_HD SegWalk(const Params& p, int64_t b, int64_t G)
     {
         Kc = p.Kc;
         const int64_t T = p.TM * p.TN;
@@ -156,7 +156,7 @@ struct SegWalk {
             start_own();
         }
     }
-    __device__ void start_own()
+    SHERRY_HD void start_own()
     {
         if (r1_tile < r1_end_tile) {
             range = 1;
@@ -167,9 +167,9 @@ struct SegWalk {
             range = 2;
         }
     }
-    __device__ bool done() const { return range == 2; }
-    __device__ bool complete() const { return cb == 0 && ce == Kc; }
-    __device__ void next()
+    SHERRY_HD bool done() const { return range == 2; }
+    SHERRY_HD bool complete() const { return cb == 0 && ce == Kc; }
+    SHERRY_HD void next()
     {
         if (range == 0) {
             const int64_t u = tile * Kc + ce;
@@ -188,7 +188,7 @@ struct SegWalk {
 
 // First and last CTA of a split tile t (one of the last R tiles): the owners
 // of its first and last unit among the G shares of the split units.
-__device__ __forceinline__ void split_owners(const Params& p, int64_t t, int64_t G, int64_t* bf, int64_t* bl)
+SHERRY_HD inline void split_owners(const Params& p, int64_t t, int64_t G, int64_t* bf, int64_t* bl)
 {
     const int64_t T = p.TM * p.TN;
     const int64_t R = T - (T / G) * G;
