@@ -470,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;                 // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;          // row within the 128-row tile
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-        const uint8_t* tbl = reinterpret_cast<const uint8_t*>(table);
+        // 128-byte aligned: a code's entry address is (code * 4) | table_s
+        const uint32_t table_s = ptx::smem_u32(table);
         int s = 0, a = 0;
         uint32_t sph = 0, aph = 0;
         int turn = 0;                               // iteration index modulo kDecGroups
@@ -519,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         else if (off == 1) v = w[j][wi] << 1;
                         else if (off <= 27) v = w[j][wi] >> (off - 2);
                         else v = __funnelshift_r(w[j][wi], w[j][wi + 1], off - 2);
-                        a_vals[g] = *reinterpret_cast<const uint32_t*>(tbl + (v & 0x7Cu));
+                        a_vals[g] = ptx::lds_u32_nv((v & 0x7Cu) | table_s);
                     }
                     ptx::tmem_st_32x32b_x32(lane_base + (uint32_t)(C::kACol0 + a * C::kACols + 32 * j), a_vals);
                 }
