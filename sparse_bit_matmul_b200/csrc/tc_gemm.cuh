@@ -472,6 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         // 128-byte aligned: a code's entry address is (code * 4) | table_s
         const uint32_t table_s = ptx::smem_u32(table);
+        // byte offsets of this row's five code words within a chunk
+        uint32_t wpos[SHERRY_CHUNK_WORDS];
+#pragma unroll
+        for (int k = 0; k < SHERRY_CHUNK_WORDS; ++k) wpos[k] = 4u * (uint32_t)sherry_word_pos(k, row);
         int s = 0, a = 0;
         uint32_t sph = 0, aph = 0;
         int turn = 0;                               // iteration index modulo kDecGroups
@@ -490,14 +494,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     quit = true;
                     break;
                 }
-                const uint32_t* codes =
-                    reinterpret_cast<const uint32_t*>(smem + C::kOffCodes + s * C::kCodeStageBytes);
+                const uint32_t codes_s = sbase + (uint32_t)(C::kOffCodes + s * C::kCodeStageBytes);
                 uint32_t w[SC][SHERRY_CHUNK_WORDS];
 #pragma unroll
                 for (int j = 0; j < SC; ++j)
 #pragma unroll
                     for (int k = 0; k < SHERRY_CHUNK_WORDS; ++k)
-                        w[j][k] = (j < nch) ? codes[j * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS) + sherry_word_pos(k, row)] : 0u;
+                        w[j][k] = (j < nch) ? ptx::lds_u32(codes_s + (uint32_t)(j * kChunkCodeBytes) + wpos[k]) : 0u;
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(empty_bar(s));
                 ok = ptx::mbar_wait_bounded(aempty_bar(a), aph ^ 1u, kWaitLimitNs);
