@@ -211,6 +211,28 @@ int device_info(DeviceInfo* out)
 }
 
 // Zero-initialised per-device workspace of at least `bytes`, ordered on `stream`.
+// CTAs of a tensor-core launch with T output tiles of BN tokens and Kc K
+// chunks each (U = T * Kc units).
+// T >= SMs: one CTA per SM (whole tiles plus an even share of the leftover
+// tiles, split across CTAs; their sums overlap the whole tiles).
+// T < SMs: the sums of split tiles come at the end of the kernel, where they
+// were measured at ~18 us for 128-token tiles (2 + 16 * BN / 128 us is the
+// estimate used here), against ~0.27 us per K chunk walked.  So every tile is
+// split into S = SMs div T equal K shares (T * S CTAs) only when that saves
+// more chunk time than the sums cost; otherwise S = 1: one CTA per tile, no
+// tile split, no cross-CTA sum.
+int64_t tc_grid(int64_t T, int64_t U, int64_t sms, int64_t Kc, int bn)
+{
+    int64_t g = sms;
+    if (T < sms) {
+        const int64_t S = sms / T;
+        const double saved_us = 0.27 * (double)Kc * (1.0 - 1.0 / (double)S);
+        const double sums_us = 2.0 + 16.0 * (double)bn / 128.0;
+        g = (S > 1 && saved_us > sums_us) ? T * S : T;
+    }
+    return std::min<int64_t>(g, U);
+}
+
 int get_workspace(size_t bytes, cudaStream_t stream, void** out)
 {
     int dev = 0;
@@ -296,7 +318,7 @@ int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alp
     p.TN = sherry_row_tiles(N);
     p.Kc = sherry_k_chunks(K);
     p.U = p.TM * p.TN * p.Kc;
-    const int64_t grid = std::min<int64_t>(di.sms, p.U);
+    const int64_t grid = tc_grid(p.TM * p.TN, p.U, di.sms, p.Kc, BN);
     void* ws = nullptr;
     const size_t ws_acc = (size_t)grid * BN * SHERRY_TILE_ROWS * sizeof(int32_t);
     st = get_workspace(ws_acc + (size_t)grid * sizeof(uint32_t), stream, &ws);
@@ -564,7 +586,7 @@ int launch_tc_noalloc(const int8_t* x, const float* xs, const void* wn, const fl
     p.TN = sherry_row_tiles(N);
     p.Kc = sherry_k_chunks(K);
     p.U = p.TM * p.TN * p.Kc;
-    const int64_t grid = std::min<int64_t>(std::min<int64_t>(di.sms, p.U), kNoAllocMaxCtas);
+    const int64_t grid = std::min<int64_t>(tc_grid(p.TM * p.TN, p.U, di.sms, p.Kc, BN), kNoAllocMaxCtas);
     p.ws = scratch;
     p.counters = reinterpret_cast<uint32_t*>(scratch + kNoAllocAccWords);
     p.status = device_status_ptr();

@@ -1,6 +1,7 @@
 // Host-side check of the tensor-core kernel's work split (SegWalk and
 // split_owners, compiled from the kernel's own header for the host): for many
-// tile counts, chunk counts and grid sizes, every (tile, K chunk) unit is
+// tile counts, chunk counts and grid sizes (one CTA per SM, and T * (SMs div
+// T) CTAs when there are fewer tiles T than SMs), every (tile, K chunk) unit is
 // walked by exactly one CTA, the CTAs' unit counts differ by at most one,
 // segments stay inside one tile, and for every tile walked by more than one
 // CTA the owner range [bf, bl] is exactly its set of contributors, with a
@@ -18,14 +19,14 @@ using sherry::tc::Params;
 using sherry::tc::SegWalk;
 using sherry::tc::split_owners;
 
-static int check(int64_t TM, int64_t TN, int64_t Kc, int64_t sms)
+static int check(int64_t TM, int64_t TN, int64_t Kc, int64_t G0)
 {
     Params p{};
     p.TM = TM;
     p.TN = TN;
     p.Kc = Kc;
     p.U = TM * TN * Kc;
-    const int64_t G = sms < p.U ? sms : p.U;
+    const int64_t G = G0 < p.U ? G0 : p.U;
     std::vector<int64_t> owner(p.U, -1);
     int64_t lo = INT64_MAX, hi = 0;
     for (int64_t b = 0; b < G; ++b) {
@@ -90,8 +91,12 @@ int main()
         for (int64_t TN : tns)
             for (int64_t Kc : kcs)
                 for (int64_t sms : smss) {
+                    // one CTA per SM, and the launch's grid for few tiles:
+                    // T * (SMs div T) when T < SMs
+                    const int64_t T = TM * TN;
                     if (check(TM, TN, Kc, sms)) return 1;
-                    ++n;
+                    if (T < sms && check(TM, TN, Kc, T * (sms / T))) return 1;
+                    n += T < sms ? 2 : 1;
                 }
     std::printf("ok %d shapes\n", n);
     return 0;
