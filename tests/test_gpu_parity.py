@@ -119,7 +119,10 @@ SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 5
          # of one chunk (one split unit), 150 tiles of five chunks (split
          # units fewer than CTAs), 200 tiles of eight chunks (split units
          # shared out by floor division)
-         (100, 19072, 128), (300, 6400, 640), (520, 5120, 1024)]
+         (100, 19072, 128), (300, 6400, 640), (520, 5120, 1024),
+         # fewer tiles than SMs with long K: every tile split into equal K
+         # shares over many CTAs (128- and 64-token tiles)
+         (130, 384, 14336), (40, 256, 14336)]
 
 
 def _kernel_serves(kernel: str, M: int, K: int) -> bool:
