@@ -347,12 +347,14 @@ def run_gpu(args, world, rank, local):
     # otherwise sherry_quant_act + the named GEMM kernel, two launches
     fused = kernel == "auto"
 
-    def layer(L):
+    def layer(L, x=None, y=None):
+        x = L["x"] if x is None else x
+        y = L["y"] if y is None else y
         if fused:
-            sbm.linear(L["x"], L["native"], L["alpha"], L["N"], out=L["y"])
+            sbm.linear(x, L["native"], L["alpha"], L["N"], out=y)
         else:
-            sbm.quant_act(L["x"], L["q"], L["s"])
-            sbm.gemm(L["q"], L["s"], L["native"], L["alpha"], L["N"], out=L["y"], kernel=kernel)
+            sbm.quant_act(x, L["q"], L["s"])
+            sbm.gemm(L["q"], L["s"], L["native"], L["alpha"], L["N"], out=y, kernel=kernel)
 
     def step():
         for L in layers:
@@ -372,7 +374,31 @@ def run_gpu(args, world, rank, local):
             sbm.quant_act(L["x"], L["q"], L["s"])
             sbm.gemm(L["q"], L["s"], L["native"], L["alpha"], L["N"], out=L["y"])
 
+    # end to end, the step's inputs and outputs each in one pinned host
+    # buffer: one H2D copy of all layer inputs, the layer calls on device
+    # views of one input and one output buffer, one D2H copy of all outputs
+    x_total = sum(L["x"].numel() for L in layers)
+    y_total = sum(L["y"].numel() for L in layers)
+    X_host = torch.empty(x_total, dtype=torch.float32).pin_memory()
+    Y_host = torch.empty(y_total, dtype=torch.float32).pin_memory()
+    X_dev = torch.empty(x_total, dtype=torch.float32, device=device)
+    Y_dev = torch.empty(y_total, dtype=torch.float32, device=device)
+    xo = yo = 0
+    for L in layers:
+        nx, ny = L["x"].numel(), L["y"].numel()
+        X_host[xo:xo + nx].copy_(L["x_host"].reshape(-1))
+        L["x_step"] = X_dev[xo:xo + nx].view(L["x"].shape)
+        L["y_step"] = Y_dev[yo:yo + ny].view(L["y"].shape)
+        xo += nx
+        yo += ny
+
     def e2e_step():
+        X_dev.copy_(X_host, non_blocking=True)
+        for L in layers:
+            layer(L, L["x_step"], L["y_step"])
+        Y_host.copy_(Y_dev, non_blocking=True)
+
+    def e2e_per_layer_step():
         for L in layers:
             L["x"].copy_(L["x_host"], non_blocking=True)
             layer(L)
@@ -385,6 +411,7 @@ def run_gpu(args, world, rank, local):
     g_quant = capture(quant_only)
     g_two = capture(two_launch_step) if fused else None
     g_e2e = capture(e2e_step)
+    g_e2e_layer = capture(e2e_per_layer_step)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -395,6 +422,7 @@ def run_gpu(args, world, rank, local):
     t_quant = max_over_ranks(time_graph(g_quant, args.steps, args.warmup, world), world)
     t_two = max_over_ranks(time_graph(g_two, args.steps, args.warmup, world), world) if fused else None
     t_e2e = max_over_ranks(time_graph(g_e2e, args.steps, args.warmup, world), world)
+    t_e2e_layer = max_over_ranks(time_graph(g_e2e_layer, args.steps, args.warmup, world), world)
     assert sbm.last_device_status() == 0, "a kernel reported a bounded wait running out"
 
     peaks, peak_src = load_peaks()
@@ -444,12 +472,16 @@ def run_gpu(args, world, rank, local):
         },
         "e2e": {"value": round(step_bytes * world * args.steps / t_e2e / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "path": ("pinned host x -> H2D -> " + ("sherry_linear" if fused else "sherry_quant_act -> "
-                         f"sherry_gemm[{kernel}]") + " -> D2H y, per layer, in one CUDA graph per step")},
+                "path": ("one pinned host buffer of the step's layer inputs -> one H2D copy -> "
+                         + ("sherry_linear" if fused else f"sherry_quant_act -> sherry_gemm[{kernel}]")
+                         + " per layer on device views -> one D2H copy of the step's outputs, "
+                         "in one CUDA graph per step"),
+                "per_layer_copies_gbs": round(step_bytes * world * args.steps / t_e2e_layer / 1e9, 2),
+                "per_layer_copies_path": "H2D of x, the layer call, D2H of y, around every layer call"},
         "gpu_launches": (1 if fused else 2) * n_launch * args.steps,
         "clocks": clocks,
     }
-    del g_step, g_gemm, g_quant, g_two, g_e2e
+    del g_step, g_gemm, g_quant, g_two, g_e2e, g_e2e_layer
     if not args.no_extras:
         out["extra"] = extras(args, layers, kernel, peaks, peak_src, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
