@@ -402,6 +402,9 @@ int launch_gemv(const int8_t* x, const float* xs, const void* wn, const float* a
         cudaFuncSetAttribute(gemv::sherry_gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
             cudaSuccess)
         return SHERRY_ERR_CUDA;
+    if (cudaFuncSetAttribute(gemv::sherry_gemv_kernel<MT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        return SHERRY_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.TN, (unsigned)NS);
     cfg.blockDim = dim3(gemv::kThreads);
@@ -477,9 +480,18 @@ int launch_decode(const decode::Params& p0, cudaStream_t stream)
     if (pl.smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
+    // One shared-memory carveout for every shape: left to the driver, the
+    // L1/shared split follows each launch's request, and consecutive layers
+    // of different shapes (27, 70 and 88 KB) then cannot share an SM, so the
+    // next layer's CTAs lose their early start (measured: 11.2 us per call
+    // alternating two shapes that take 7.6 and 9.0 us on their own).
     std::call_once(attr_once, [&] {
         attr_err = cudaFuncSetAttribute(decode::sherry_decode_kernel<MT, FUSED>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, decode::kSmemBudget);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(decode::sherry_decode_kernel<MT, FUSED>,
+                                            cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            cudaSharedmemCarveoutMaxShared);
     });
     if (attr_err != cudaSuccess) return SHERRY_ERR_CUDA;
     return cuda_status(launch_pdl(decode::sherry_decode_kernel<MT, FUSED>, dim3((unsigned)pl.G),
