@@ -239,6 +239,29 @@ __device__ __forceinline__ void mma_i8_ts_elect(uint32_t d_tmem, uint32_t a_tmem
         : "memory");
 }
 
+// One K chunk of MMAs (four K=32 steps) from a converged warp: one
+// elect.sync for the four, the accumulate flag of the first step given,
+// the other three always accumulating.  a_tmem: the chunk's first A column;
+// b_desc: the descriptor of its first K step (each step adds 32 bytes, 2 in
+// the descriptor's 16-byte address units).
+__device__ __forceinline__ void mma_i8_ts_chunk_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                      uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e, t;\n\t.reg .b32 a1, a2, a3;\n\t.reg .b64 b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, %4, %4;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+        "add.u64 b1, %2, 2;\n\tadd.u64 b2, %2, 4;\n\tadd.u64 b3, %2, 6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [a1], b1, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [a2], b2, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [a3], b3, %3, t;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void tc_commit_elect(uint32_t bar)
 {
     asm volatile(

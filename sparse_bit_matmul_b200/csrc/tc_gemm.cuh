@@ -430,19 +430,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (left >= SC) {
 #pragma unroll
                     for (int j = 0; j < SC; ++j)
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            ptx::mma_i8_ts_elect(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
-                                                 desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
-                                                 (j == 0 && ks == 0) ? acc0 : 1u);
+                        ptx::mma_i8_ts_chunk_elect(d_tmem, a_tmem + (uint32_t)(32 * j),
+                                                   desc0 + (uint64_t)((j * C::kBChunkBytes) >> 4), C::kIdesc,
+                                                   j == 0 ? acc0 : 1u);
                     left -= SC;
                 } else {
                     for (int j = 0; j < left; ++j)
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            ptx::mma_i8_ts_elect(d_tmem, a_tmem + (uint32_t)(32 * j + 8 * ks),
-                                                 desc0 + (uint64_t)((j * C::kBChunkBytes + 32 * ks) >> 4), C::kIdesc,
-                                                 (j == 0 && ks == 0) ? acc0 : 1u);
+                        ptx::mma_i8_ts_chunk_elect(d_tmem, a_tmem + (uint32_t)(32 * j),
+                                                   desc0 + (uint64_t)((j * C::kBChunkBytes) >> 4), C::kIdesc,
+                                                   j == 0 ? acc0 : 1u);
                     left = 0;
                 }
                 ptx::tc_commit_elect(empty_bar(s));
