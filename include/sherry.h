@@ -132,17 +132,22 @@ int sherry_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_i8, float* 
 #define SHERRY_GEMV_MAX_M 4
 /* Largest M of the decode kernel, sherry_gemm_decode. */
 #define SHERRY_DECODE_MAX_M 8
-/* Largest M for which sherry_linear is a single fused launch. */
-#define SHERRY_LINEAR_FUSED_MAX_M 4
+/* Largest M for which sherry_gemm chooses the decode kernel: measured on
+ * B200 over the (4096,4096), (4096,14336), (14336,4096) projections, the
+ * tensor-core kernel is faster from M = 3 on. */
+#define SHERRY_GEMM_DECODE_AUTO_MAX_M 2
+/* Largest M for which sherry_linear is a single fused launch (quantiser and
+ * decode kernel); from M = 2 on the two-launch path measured faster. */
+#define SHERRY_LINEAR_FUSED_MAX_M 1
 
 /*
  * sherry_gemm -- device, asynchronous.  y = epilogue(x_i8 . T^T) (sec. 2.2
  * steps 2-4): exact int32 accumulation, then
  * y[m][n] = (float)((float)acc * alpha[n]) * x_scale[m].
- * M <= SHERRY_DECODE_MAX_M runs sherry_gemm_decode (when a CTA's share of
- * the codes fits in shared memory, i.e. K up to about 600000 weights), any
- * other shape sherry_gemm_tc (tensor cores); all kernels give identical
- * results.
+ * M <= SHERRY_GEMM_DECODE_AUTO_MAX_M runs sherry_gemm_decode (when a CTA's
+ * share of the codes fits in shared memory, i.e. K up to about 600000
+ * weights), any other shape sherry_gemm_tc (tensor cores); all kernels give
+ * identical results.
  *   x_i8     [in]  int8 [M][K], device memory, 16-byte aligned
  *   x_scale  [in]  fp32 [M], device memory
  *   Wnative  [in]  kernel-native codes from sherry_repack, device memory, 16-byte aligned
@@ -200,9 +205,9 @@ int sherry_gemm_decode(const int8_t* x_i8, const float* x_scale, const void* Wna
  * sherry_linear -- device, asynchronous.  The whole online step of the page
  * (sec. 2.2 steps 1-4) from fp32 activations: the sherry_quant_act rule
  * followed by the sherry_gemm contraction and epilogue, with bit-identical
- * results.  For M <= SHERRY_LINEAR_FUSED_MAX_M it is one launch of the
- * decode kernel that also quantises (every CTA reads the whole activation
- * rows, takes their absmax and quantises them into its shared memory).
+ * results.  For M <= SHERRY_LINEAR_FUSED_MAX_M (one token) it is one launch
+ * of the decode kernel that also quantises (every CTA reads the whole
+ * activation row, takes its absmax and quantises it into its shared memory).
  * Other shapes run sherry_quant_act into a per-device buffer of the library
  * (allocated on first use, grown with a stream synchronisation) and then
  * sherry_gemm.

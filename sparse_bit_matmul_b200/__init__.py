@@ -147,7 +147,8 @@ def quant_act(x, out_q=None, out_s=None):
 
 GEMV_MAX_M = 4      # SHERRY_GEMV_MAX_M
 DECODE_MAX_M = 8    # SHERRY_DECODE_MAX_M
-LINEAR_FUSED_MAX_M = 4   # SHERRY_LINEAR_FUSED_MAX_M
+GEMM_DECODE_AUTO_MAX_M = 2   # SHERRY_GEMM_DECODE_AUTO_MAX_M
+LINEAR_FUSED_MAX_M = 1   # SHERRY_LINEAR_FUSED_MAX_M
 
 
 def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: bool = True,
@@ -187,7 +188,7 @@ def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: boo
 
 def linear(x, w_native, alpha, N: int, out=None, acc=None, out_q=None, out_s=None, want_y: bool = True):
     """y fp32 [M][N] straight from fp32 activations x [M][K] (sherry_linear:
-    quantiser + GEMM, one launch for M <= 4).  Optional acc int32 [M][N] and
+    quantiser + GEMM, one launch for M = 1).  Optional acc int32 [M][N] and
     out_q int8 [M][K] / out_s fp32 [M] receive the exact accumulators and the
     quantised activations."""
     import torch

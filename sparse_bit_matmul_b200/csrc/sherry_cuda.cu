@@ -660,7 +660,7 @@ int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnativ
 {
     int st = check_gemm_args(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K);
     if (st != SHERRY_OK) return st;
-    if (M <= SHERRY_DECODE_MAX_M) {
+    if (M <= SHERRY_GEMM_DECODE_AUTO_MAX_M) {
         DeviceInfo di;
         st = device_info(&di);
         if (st != SHERRY_OK) return st;
@@ -720,9 +720,8 @@ int sherry_linear_ex(const float* x, const void* Wnative, const float* alpha, fl
             p.M = M;
             p.N = N;
             p.K = K;
-            if (M == 1) return launch_decode<1, true>(p, s);
-            if (M == 2) return launch_decode<2, true>(p, s);
-            return launch_decode<4, true>(p, s);
+            static_assert(SHERRY_LINEAR_FUSED_MAX_M == 1, "fused launches instantiated for one token");
+            return launch_decode<1, true>(p, s);
         }
     }
     if (!x_i8) {
