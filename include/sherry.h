@@ -270,7 +270,9 @@ int sherry_gemm_simt(const int8_t* x_i8, const float* x_scale, const void* Wnati
  * scratch array compiled into the library: 2.6 MB, reserved on every GPU
  * that loads the library until the process exits.  It therefore serves
  * decode shapes only: M <= 32 tokens, otherwise SHERRY_ERR_UNSUPPORTED_SHAPE
- * is returned before anything is launched.  It calls no cudaMalloc or
+ * is returned before anything is launched.  For M <=
+ * SHERRY_GEMM_DECODE_AUTO_MAX_M it runs the decode kernel, which needs no
+ * scratch at all, as sherry_gemm would.  It calls no cudaMalloc or
  * cudaFree.  Each call first clears (cudaMemsetAsync on `stream`) the part
  * of the scratch it uses.
  * The first call on a device looks up the scratch's device address with that

@@ -798,6 +798,15 @@ int sherry_gemm_noalloc(const int8_t* x_i8, const float* x_scale, const void* Wn
     if (st != SHERRY_OK) return st;
     if (M > kNoAllocMaxBN) return SHERRY_ERR_UNSUPPORTED_SHAPE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the decode kernel needs no workspace at all: the same choice as sherry_gemm
+    if (M <= SHERRY_GEMM_DECODE_AUTO_MAX_M) {
+        DeviceInfo di;
+        st = device_info(&di);
+        if (st != SHERRY_OK) return st;
+        DecodePlan pl;
+        if (decode_plan(N, sherry_k_chunks(K), M, di.sms, &pl))
+            return sherry_gemm_decode(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
+    }
     if (M <= 16) return launch_tc_noalloc<16, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
     return launch_tc_noalloc<32, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
 }
