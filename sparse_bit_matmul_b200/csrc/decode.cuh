@@ -216,8 +216,11 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             if (lane == 0) warp_max[(m & 1) * 16 + warp] = mx;
             __syncthreads();
-            float a = 0.0f;
-            for (int w = 0; w < nwarps; ++w) a = fmaxf(a, warp_max[(m & 1) * 16 + w]);
+            // every warp combines the (at most 16) warp maxima: one load per
+            // lane and a shuffle tree, not a chain of dependent loads
+            float a = lane < nwarps ? warp_max[(m & 1) * 16 + lane] : 0.0f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
             const quant::Scale sc = quant::make_scale(a);
             if (tid == 0) {
                 scale_s[m] = sc.s;
