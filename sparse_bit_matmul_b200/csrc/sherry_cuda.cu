@@ -297,6 +297,26 @@ unsigned* device_status_ptr()
     return static_cast<unsigned*>(p);
 }
 
+// Launch with programmatic dependent launch: the kernel may start while the
+// previous kernel on the stream finishes; it orders itself with
+// griddepcontrol.wait before touching anything that kernel may write.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int BN, int SC>
 int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y, int32_t* acc,
               int64_t M, int64_t N, int64_t K, cudaStream_t stream)
@@ -342,29 +362,12 @@ int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alp
     cudaError_t e = cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN, SC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return SHERRY_ERR_CUDA;
-    tc::sherry_gemm_tc_kernel<BN, SC><<<(unsigned)grid, tc::kThreads, smem, stream>>>(map, ymap, p);
+    e = launch_pdl(tc::sherry_gemm_tc_kernel<BN, SC>, dim3((unsigned)grid), dim3(tc::kThreads), (size_t)smem,
+                   stream, map, ymap, p);
+    if (e != cudaSuccess) return cuda_status(e);
     return cuda_status(cudaGetLastError());
 }
 
-// Launch with programmatic dependent launch: the kernel may start while the
-// previous kernel on the stream finishes; it orders itself with
-// griddepcontrol.wait before touching anything that kernel may write.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       Args... args)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
 
 template <int MT>
 int launch_gemv(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y, int32_t* acc,
@@ -619,7 +622,9 @@ int launch_tc_noalloc(const int8_t* x, const float* xs, const void* wn, const fl
     if (cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN, SC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return SHERRY_ERR_CUDA;
-    tc::sherry_gemm_tc_kernel<BN, SC><<<(unsigned)grid, tc::kThreads, smem, stream>>>(map, ymap, p);
+    const cudaError_t e = launch_pdl(tc::sherry_gemm_tc_kernel<BN, SC>, dim3((unsigned)grid), dim3(tc::kThreads),
+                                     (size_t)smem, stream, map, ymap, p);
+    if (e != cudaSuccess) return cuda_status(e);
     return cuda_status(cudaGetLastError());
 }
 

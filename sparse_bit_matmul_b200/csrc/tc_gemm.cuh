@@ -323,11 +323,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // Programmatic dependent launch: everything above (barriers, tensor
+    // memory, table) overlaps the end of the previous kernel on the stream.
+    // The roles that touch global memory the previous kernel may write or
+    // read (the producer: activations; the epilogue: scales, y, acc and the
+    // split-K workspace) wait for it to complete; the decoders and the MMA
+    // warp only use this CTA's shared and tensor memory.
+    ptx::pdl_launch_dependents();
 
     if (warp == kProducerWarp) {
         // Converged warp, elected-lane issue and a non-blocking test of the
         // next slot, for the same reason as the MMA loop below: a copy issued
         // late delays every role after it.
+        ptx::pdl_wait();
         int s = 0;
         uint32_t ph = 0;
         bool ready = false;                      // empty(s) already seen complete
@@ -533,6 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
     } else if (warp >= kEpiWarp0) {
+        ptx::pdl_wait();
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
