@@ -229,3 +229,41 @@ def test_config0_tiny_exact():
         y, acc, _, _ = run_gpu(x, native, alpha_d, 128, kernel)
         assert np.array_equal(acc, acc_o)
         assert np.array_equal(y, y_o)
+
+
+# ------------------------------------------------- layers chained on one stream
+@pytest.mark.parametrize("route", ["linear", "quant+gemm", "quant+tc"])
+@pytest.mark.parametrize("M", [1, 2, 8, 64])
+def test_chained_layers_one_stream(M, route):
+    """Six layers, each fed the previous layer's output, queued on one stream
+    with no synchronisation in between: the kernels start early under
+    programmatic dependent launch, so a read of the activations before the
+    previous layer finished would show here.  Each layer must equal the
+    oracle applied to the device's own previous output."""
+    K = N = 1024
+    L = 6
+    Ws = [synth.weights(7, i, N, K) for i in range(L)]
+    ups = [upload_weights(W) for W in Ws]
+    x0 = synth.activations(7, 0, M, K)
+    xd = torch.from_numpy(x0).cuda()
+    ys, accs = [], []
+    cur = xd
+    for i, (native, alpha_d, _, _) in enumerate(ups):
+        y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+        if route == "linear":
+            sbm.linear(cur, native, alpha_d, N, out=y, acc=acc)
+        else:
+            q, s = sbm.quant_act(cur)
+            sbm.gemm(q, s, native, alpha_d, N, out=y, acc=acc, kernel="tc" if route == "quant+tc" else "auto")
+        ys.append(y)
+        accs.append(acc)
+        cur = y
+    torch.cuda.synchronize()
+    prev = x0
+    for i in range(L):
+        y_o, acc_o, *_ = oracle.reference(prev, Ws[i])
+        assert np.array_equal(accs[i].cpu().numpy(), acc_o), f"layer {i}"
+        y_i = ys[i].cpu().numpy()
+        assert_y_close(y_i, y_o)
+        prev = y_i
