@@ -1,5 +1,6 @@
-// Inline-PTX wrappers for sm_100a: mbarriers, bulk/tensor copies (TMA, no
-// multicast), tcgen05 tensor-memory and MMA instructions.
+// Inline-PTX wrappers for sm_100a: mbarriers, bulk/tensor copies (TMA, into
+// this CTA's own shared memory only), tcgen05 tensor-memory and MMA
+// instructions.
 #pragma once
 
 #include <cstdint>
