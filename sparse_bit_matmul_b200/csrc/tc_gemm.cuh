@@ -32,12 +32,13 @@
 // of SC * 2560 bytes of codes, SC 2D TMA boxes of activations, SC * 4 MMAs),
 // so that the fixed cost of a stage's barriers is paid once per SC chunks.
 //
-// Warp roles (576 threads):
+// Warp roles (576 threads; 448 for 192-token tiles, which have two decoder
+// groups):
 //   warp 0       producer: per stage one bulk copy of the codes and one 2D
 //                TMA of the activation tile per chunk
-//   warp 1       TMEM allocation and MMA issue (one thread)
+//   warp 1       TMEM allocation and MMA issue (an elected lane)
 //   warps 2-13   three decoder groups of four warps (each group covers the
-//                four TMEM lane quadrants), taking K chunks in turn
+//                four TMEM lane quadrants), taking stages in turn
 //   warps 14-17  epilogue (one warp per lane quadrant)
 // Loop indices (stage, phase, tile coordinates) advance incrementally: no
 // integer division on the per-chunk path.
@@ -58,16 +59,19 @@ namespace tc {
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kDecWarp0 = 2;
-constexpr int kDecGroups = 3;
-constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;
-constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kTmemCols = 512;
 constexpr int kChunkCodeBytes = SHERRY_CHUNK_BYTES_PER_TILE;   // 2560
 constexpr uint64_t kWaitLimitNs = 2000000000ull;              // 2 s per wait
 
 template <int BN, int SC>
 struct Cfg {
-    static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
+    static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 192, "BN");
+    // 192-token tiles: two 192-column accumulators leave 128 TMEM columns,
+    // two A slots, so two decoder groups (the rings must be at least as deep
+    // as the number of groups); three groups otherwise
+    static constexpr int kDecGroups = BN == 192 ? 2 : 3;
+    static constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;
+    static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
     static_assert(SC >= 1 && SC <= 4, "SC");
     static constexpr int kBChunkBytes = BN * 128;
     static constexpr int kBStageBytes = SC * kBChunkBytes;
@@ -253,7 +257,7 @@ struct StageWalk {
 };
 
 template <int BN, int SC>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
     sherry_gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap,
                           const Params p)
 {
@@ -469,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xffffffffu, done) && lane == 0)
                 atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
         }
-    } else if (warp >= kDecWarp0 && warp < kDecWarp0 + 4 * kDecGroups) {
+    } else if (warp >= kDecWarp0 && warp < kDecWarp0 + 4 * C::kDecGroups) {
         const int grp = (warp - kDecWarp0) / 4;
         const int quad = warp & 3;                 // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;          // row within the 128-row tile
@@ -482,11 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < SHERRY_CHUNK_WORDS; ++k) wpos[k] = 4u * (uint32_t)sherry_word_pos(k, row);
         int s = 0, a = 0;
         uint32_t sph = 0, aph = 0;
-        int turn = 0;                               // iteration index modulo kDecGroups
+        int turn = 0;                               // iteration index modulo C::kDecGroups
         bool quit = false;
         SegWalk w(p, blockIdx.x, G);
         for (; !w.done() && !quit; w.next()) {
-          for (int left = (int)(w.ce - w.cb); left > 0; left -= SC, turn = (turn + 1 == kDecGroups) ? 0 : turn + 1) {
+          for (int left = (int)(w.ce - w.cb); left > 0; left -= SC, turn = (turn + 1 == C::kDecGroups) ? 0 : turn + 1) {
             const int nch = left < SC ? left : SC;
             const bool mine = turn == grp;
             if (mine) {
@@ -540,12 +544,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++a == C::kAStages) { a = 0; aph ^= 1u; }
           }
         }
-    } else if (warp >= kEpiWarp0) {
+    } else if (warp >= C::kEpiWarp0) {
         ptx::pdl_wait();
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-        const int etid = threadIdx.x - kEpiWarp0 * 32;     // 0..127
+        const int etid = threadIdx.x - C::kEpiWarp0 * 32;     // 0..127
         int64_t seg = 0;
         int d = 0;
         uint32_t dph = 0;
