@@ -122,7 +122,9 @@ SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 5
          (100, 19072, 128), (300, 6400, 640), (520, 5120, 1024),
          # fewer tiles than SMs with long K: every tile split into equal K
          # shares over many CTAs (128- and 64-token tiles)
-         (130, 384, 14336), (40, 256, 14336)]
+         (130, 384, 14336), (40, 256, 14336),
+         # 192-token tiles (M >= 1536), the last one ragged
+         (1600, 300, 512)]
 
 
 def _kernel_serves(kernel: str, M: int, K: int) -> bool:
