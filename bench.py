@@ -534,7 +534,7 @@ def extras(args, layers, kernel, peaks, peak_src, world):
         small[str(M)] = round(nb * max(3, args.steps // 4) / t / 1e9, 2)
         del g
     res["small_batch_decode_gbs"] = small
-    res["small_batch_step"] = ("sherry_quant_act + sherry_gemm (decode kernel for M <= 8, tensor cores above) "
+    res["small_batch_step"] = ("sherry_quant_act + sherry_gemm (decode kernel for M <= 2, tensor cores above) "
                                "per layer call"
                                if kernel == "auto" else f"GEMM kernel {kernel} only")
     # prefill GEMM, M = 2048 (L2 flushed between timed launches)
