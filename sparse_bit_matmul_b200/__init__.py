@@ -155,7 +155,7 @@ def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: boo
          kernel: str = "auto"):
     """y fp32 [M][N] (and optionally exact int32 acc) from int8 activations and
     kernel-native codes.  kernel: "auto" (sherry_gemm: the decode kernel
-    for M <= 8, tensor cores above), "decode", "tc", "gemv" (the page's
+    for M <= 2, tensor cores above), "decode", "tc", "gemv" (the page's
     table lookup), "simt" (comparison kernel) or "noalloc"."""
     import torch
     M, K = x_i8.shape
