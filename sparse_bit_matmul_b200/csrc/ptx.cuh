@@ -109,18 +109,8 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         : "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
-                                            uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
 // Elected-lane forms of the three copy-issue steps, for a converged warp
-// (see mma_i8_ts_elect): one lane issues, every lane runs the code.
+// (see mma_i8_ts_chunk_elect): one lane issues, every lane runs the code.
 __device__ __forceinline__ void mbar_arrive_expect_tx_elect(uint32_t bar, uint32_t bytes)
 {
     asm volatile(
@@ -203,48 +193,16 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Commit all prior tcgen05 async operations of this thread to an mbarrier.
-__device__ __forceinline__ void tc_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-
 // D[128 x N] (+)= A[128 x 32] (tensor memory, int8, K-major) x B[32 x N]
-// (shared memory descriptor, int8, K-major); int32 accumulators.
-__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate)
-{
-    uint32_t z = 0;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z)
-        : "memory");
-}
-
-// As mma_i8_ts and tc_commit, executed by a whole converged warp: one lane,
+// (shared memory descriptor, int8, K-major), int32 accumulators, for one K
+// chunk (four K=32 steps), executed by a whole converged warp: one lane,
 // chosen by elect.sync inside the instruction sequence, issues.  With every
 // lane running the issue loop the compiler sees the operands as warp-uniform
-// and keeps them in uniform registers, so consecutive MMAs issue back to back.
-__device__ __forceinline__ void mma_i8_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// One K chunk of MMAs (four K=32 steps) from a converged warp: one
-// elect.sync for the four, the accumulate flag of the first step given,
-// the other three always accumulating.  a_tmem: the chunk's first A column;
-// b_desc: the descriptor of its first K step (each step adds 32 bytes, 2 in
-// the descriptor's 16-byte address units).
+// and keeps them in uniform registers, so consecutive MMAs issue back to
+// back.  The accumulate flag of the first step is given, the other three
+// always accumulate.  a_tmem: the chunk's first A column; b_desc: the
+// descriptor of its first K step (each step adds 32 bytes, 2 in the
+// descriptor's 16-byte address units).
 __device__ __forceinline__ void mma_i8_ts_chunk_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                                       uint32_t idesc, uint32_t accumulate)
 {
@@ -263,6 +221,8 @@ __device__ __forceinline__ void mma_i8_ts_chunk_elect(uint32_t d_tmem, uint32_t 
         : "memory");
 }
 
+// tcgen05.commit (arrive on `bar` when this thread's MMAs so far complete),
+// from a converged warp, one elected lane issuing.
 __device__ __forceinline__ void tc_commit_elect(uint32_t bar)
 {
     asm volatile(
@@ -351,12 +311,6 @@ __device__ __forceinline__ void cluster_wait_acquire()
 {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ uint32_t cluster_ctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
 // Address of `local_addr`'s counterpart in the shared memory of cluster CTA `cta`.
 __device__ __forceinline__ uint32_t mapa(uint32_t local_addr, uint32_t cta)
 {
@@ -386,12 +340,5 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
-__device__ __forceinline__ uint2 lds_u64(uint32_t addr)
-{
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-    return v;
-}
-
 }  // namespace ptx
 }  // namespace sherry
