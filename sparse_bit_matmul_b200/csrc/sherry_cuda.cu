@@ -759,10 +759,12 @@ int sherry_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* Wnative
     if (M <= 32) return launch_tc<32, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
     if (M <= 64) return launch_tc<64, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
     // 192-token tiles decode each weight tile for 1.5x the tokens; measured
-    // faster from M ~ 1536 on (M=2048: 115.5 -> 111.5 us, M=8192: 407 -> 396
+    // faster from M ~ 1536 on (M=2048: 115.5 -> 111.5 us, M=8192: 407 -> 380
     // us at K=4096, N=14336), slower where their padding is large (M=1024).
+    // One-chunk stages: four A slots and three decoder groups beat two-chunk
+    // stages with two (M=8192: 398 -> 380 us, K=14336 -> N=4096: 99 -> 96.5).
     if (M < 1536) return launch_tc<128, 2>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
-    return launch_tc<192, 2>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+    return launch_tc<192, 1>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
 }
 
 int sherry_gemm_gemv(const int8_t* x_i8, const float* x_scale, const void* Wnative, const float* alpha, float* y,

@@ -32,8 +32,8 @@
 // of SC * 2560 bytes of codes, SC 2D TMA boxes of activations, SC * 4 MMAs),
 // so that the fixed cost of a stage's barriers is paid once per SC chunks.
 //
-// Warp roles (576 threads; 448 for 192-token tiles, which have two decoder
-// groups):
+// Warp roles (576 threads; 448 for 192-token tiles with two-chunk stages,
+// which have two decoder groups):
 //   warp 0       producer: per stage one bulk copy of the codes and one 2D
 //                TMA of the activation tile per chunk
 //   warp 1       TMEM allocation and MMA issue (an elected lane)
@@ -66,10 +66,11 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;              // 2 s per wait
 template <int BN, int SC>
 struct Cfg {
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 192, "BN");
-    // 192-token tiles: two 192-column accumulators leave 128 TMEM columns,
-    // two A slots, so two decoder groups (the rings must be at least as deep
-    // as the number of groups); three groups otherwise
-    static constexpr int kDecGroups = BN == 192 ? 2 : 3;
+    // 192-token tiles: two 192-column accumulators leave 128 TMEM columns:
+    // four one-chunk A slots (SC = 1, three decoder groups, the form used)
+    // or two two-chunk slots (SC = 2, then only two groups: the rings must be
+    // at least as deep as the number of groups)
+    static constexpr int kDecGroups = (BN == 192 && SC == 2) ? 2 : 3;
     static constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;
     static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
     static_assert(SC >= 1 && SC <= 4, "SC");
