@@ -202,10 +202,13 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             float4 v[kXV];
             float mx = 0.0f;
             if (in_regs) {
-                // unconditional loads (indices past the row repeat its last
-                // float4, which leaves the maximum unchanged): all in flight at once
+                // predicated loads, all in flight at once; slots past the row
+                // hold zeros, which leave the maximum unchanged
 #pragma unroll
-                for (int u = 0; u < kXV; ++u) v[u] = xr[min(tid + u * nthr, K4 - 1)];
+                for (int u = 0; u < kXV; ++u) {
+                    const int idx = tid + u * nthr;
+                    v[u] = idx < K4 ? xr[idx] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                }
 #pragma unroll
                 for (int u = 0; u < kXV; ++u) mx = fmaxf(mx, quant::absmax4(v[u]));
             } else {
