@@ -18,6 +18,16 @@ it restates:
   gemm_lut          sec. 2.2 steps 1-4 (16-entry segment table, sign, add)
   epilogue          sec. 2.2 step 4 (float scaling after integer sums)
 
+The second source, ``w4a8_oracle.c``, states the W4A8 FastGEMM path of the
+OdysseyLLM review page (xllm-io.github.io/paper-review/blog/odysseyllm):
+  w4a8_quantise     sec. 3.3  (per-channel symmetric int4, S = max|W| / 7;
+                    the clipping factors gamma, beta taken as 1)
+  w4a8_pack/unpack  sec. 5.2  (4-bit two's complement, two per byte)
+  w4a8_sint4_to_s8  sec. 3.2 / 5.2 (shift left by 4: the int8 value 16 w)
+  w4a8_gemm         sec. 3.1 / 5.2 (int8 contraction of q with 16 w in int32,
+                    then divided by 16)
+  w4a8_epilogue     sec. 3.1 (per-channel dequantisation after the GEMM)
+
 Parity status of each function is listed in the header of the tests that pin
 it; end to end ("is this the method") is unpinned beyond those pins because
 the page prints no output values for a Sherry matmul.
@@ -43,11 +53,12 @@ class OracleError(RuntimeError):
 
 def build(force: bool = False) -> str:
     """Compile the oracle (plain C, OpenMP over independent rows)."""
-    src = os.path.join(_HERE, "sherry_oracle.c")
-    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(src):
+    srcs = [os.path.join(_HERE, f) for f in ("sherry_oracle.c", "w4a8_oracle.c")]
+    newest = max(os.path.getmtime(f) for f in srcs)
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < newest:
         subprocess.check_call(
             ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
-             "-fno-fast-math", "-o", _SO, src, "-lm"])
+             "-fno-fast-math", "-o", _SO, *srcs, "-lm"])
     return _SO
 
 
@@ -74,6 +85,15 @@ def _load():
         L.oracle_epilogue.argtypes = [vp, vp, vp, i64, i64, vp]
         L.oracle_epilogue.restype = None
         L.oracle_forward.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
+        L.w4a8_oracle_quantise.argtypes = [vp, i64, i64, vp, vp]
+        L.w4a8_oracle_row_bytes.argtypes = [i64]
+        L.w4a8_oracle_row_bytes.restype = i64
+        L.w4a8_oracle_pack.argtypes = [vp, i64, i64, vp]
+        L.w4a8_oracle_unpack.argtypes = [vp, i64, i64, vp]
+        L.w4a8_oracle_sint4_to_s8.argtypes = [ctypes.c_int]
+        L.w4a8_oracle_gemm.argtypes = [vp, vp, i64, i64, i64, vp]
+        L.w4a8_oracle_epilogue.argtypes = [vp, vp, vp, i64, i64, vp]
+        L.w4a8_oracle_epilogue.restype = None
         _lib = L
     return _lib
 
@@ -209,3 +229,74 @@ def reference(x: np.ndarray, W: np.ndarray):
     q, s = quant_act(x)
     y, acc = forward(q, s, codes, alpha, W.shape[1])
     return y, acc, q, s, codes, alpha
+
+
+# ---- W4A8 FastGEMM (OdysseyLLM review page) ---------------------------------
+W4_NOT_MULTIPLE = 5
+
+
+def w4a8_quantise(W: np.ndarray):
+    """sec. 3.3 with gamma = beta = 1: (W_q int8 [N][K] in [-8, 7], S fp32 [N])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    Wq = np.empty((N, K), dtype=np.int8)
+    S = np.empty(N, dtype=np.float32)
+    _check(_load().w4a8_oracle_quantise(_p(W), N, K, _p(Wq), _p(S)), "w4a8_quantise")
+    return Wq, S
+
+
+def w4a8_pack(Wq: np.ndarray) -> np.ndarray:
+    """sec. 5.2: two SINT4 values per byte, even k in the low nibble."""
+    Wq = np.ascontiguousarray(Wq, dtype=np.int8)
+    N, K = Wq.shape
+    out = np.empty((N, int(_load().w4a8_oracle_row_bytes(K))), dtype=np.uint8)
+    _check(_load().w4a8_oracle_pack(_p(Wq), N, K, _p(out)), "w4a8_pack")
+    return out
+
+
+def w4a8_unpack(packed: np.ndarray, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    Wq = np.empty((N, K), dtype=np.int8)
+    _check(_load().w4a8_oracle_unpack(_p(packed), N, K, _p(Wq)), "w4a8_unpack")
+    return Wq
+
+
+def w4a8_sint4_to_s8(nibble: int) -> int:
+    """sec. 3.2 / 5.2: the 4 bits shifted into the high half of an int8."""
+    return int(_load().w4a8_oracle_sint4_to_s8(int(nibble)))
+
+
+def w4a8_gemm(q: np.ndarray, packed: np.ndarray, K: int) -> np.ndarray:
+    """sec. 3.1 / 5.2: acc = (sum_k q[m][k] * SINT4toS8(w[n][k])) / 16, int32."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    M, N = q.shape[0], packed.shape[0]
+    acc = np.empty((M, N), dtype=np.int32)
+    _check(_load().w4a8_oracle_gemm(_p(q), _p(packed), M, N, K, _p(acc)), "w4a8_gemm")
+    return acc
+
+
+def w4a8_epilogue(acc: np.ndarray, S: np.ndarray, s: np.ndarray) -> np.ndarray:
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    S = np.ascontiguousarray(S, dtype=np.float32)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    M, N = acc.shape
+    y = np.empty((M, N), dtype=np.float32)
+    _load().w4a8_oracle_epilogue(_p(acc), _p(S), _p(s), M, N, _p(y))
+    return y
+
+
+def w4a8_forward(q: np.ndarray, s: np.ndarray, packed: np.ndarray, S: np.ndarray, K: int):
+    """contract -> divide by 16 -> dequantise; returns (y, acc)."""
+    acc = w4a8_gemm(q, packed, K)
+    return w4a8_epilogue(acc, S, s), acc
+
+
+def w4a8_reference(x: np.ndarray, W: np.ndarray):
+    """The whole W4A8 path from fp32 x and W: (y, acc, q, s, packed, S)."""
+    Wq, S = w4a8_quantise(W)
+    packed = w4a8_pack(Wq)
+    q, s = quant_act(x)
+    y, acc = w4a8_forward(q, s, packed, S, W.shape[1])
+    return y, acc, q, s, packed, S
