@@ -55,9 +55,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["decode", "prefill"], default=None,
-                    help="run a few launches of one layer shape (K=4096, N=14336; M=1 or 2048) "
-                         "and exit: the target of the committed ncu captures")
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "w4a8"], default=None,
+                    help="run a few launches of one layer shape (K=4096, N=14336; M=1 or 2048; "
+                         "w4a8: the SINT4 x int8 GEMM at M=2048) and exit: the target of the "
+                         "committed ncu captures")
     return ap.parse_args(argv)
 
 
@@ -585,7 +586,71 @@ def extras(args, layers, kernel, peaks, peak_src, world):
     res["int8_library_gemm_tops"] = {"value": round(lib_tops, 1), "how": "torch._int_mm 8192^3, 10 launches"}
     for v in pre.values():
         v["frac_of_library_int8"] = round(v["int_tops_dense_equiv"] / lib_tops, 4)
+    res["w4a8"] = w4a8_extras(args, flush, int8_peak, lib_tops, world)
     return res
+
+
+def w4a8_bytes(M: int, K: int, N: int) -> int:
+    """SINT4 weights + fp32 channel scales + int8 activations + token scales."""
+    return N * K // 2 + 4 * N + M * K + 4 * M
+
+
+def w4a8_extras(args, flush, int8_peak, lib_tops, world):
+    """W4A8 FastGEMM (SINT4 weights x int8 activations) on the tensor-core
+    kernel: small M over a rotation of weight copies larger than twice L2,
+    and prefill launches after an L2 flush."""
+    import torch
+    import sparse_bit_matmul_b200 as sbm
+    import synth
+    out = {"kernel": "sherry_gemm_tc_kernel<BN, SC, int4 weights> via sherry_w4a8_gemm",
+           "weights": "synthetic N(0, 0.02) quantised per channel to SINT4 (S = max|w| / 7)"}
+    K, N = 4096, 14336
+    copies = 9                                    # 9 x 29.4 MB = 264 MB > 2 x L2
+    mats = []
+    for c in range(copies):
+        w4, scale = sbm.w4a8_pack(synth.config_weights(1, c, K, N))
+        mats.append((sbm.w4a8_repack(torch.from_numpy(w4).cuda(), N, K), torch.from_numpy(scale).cuda()))
+    small = {}
+    for M in (1, 16):
+        q, s = sbm.quant_act(torch.from_numpy(synth.config_activations(2, 0, M, K)).cuda())
+        y = torch.empty((M, N), device="cuda")
+
+        def fn():
+            for nat, sc in mats:
+                sbm.w4a8_gemm(q, s, nat, sc, N, out=y)
+        g = capture(fn)
+        reps = max(3, args.steps // 4)
+        t = max_over_ranks(time_graph(g, reps, 2, world), world)
+        gbs = w4a8_bytes(M, K, N) * copies * reps / t / 1e9
+        small[str(M)] = {"gbs": round(gbs, 1), "us_per_call": round(t / (copies * reps) * 1e6, 2)}
+        del g
+    out[f"small_M_K{K}_N{N}_rotation{copies}"] = small
+    pre = {}
+    for K, N in [(4096, 14336), (14336, 4096)]:
+        M = 2048
+        w4, scale = sbm.w4a8_pack(synth.config_weights(3, 0, K, N))
+        nat = sbm.w4a8_repack(torch.from_numpy(w4).cuda(), N, K)
+        sc = torch.from_numpy(scale).cuda()
+        q, s = sbm.quant_act(torch.from_numpy(synth.config_activations(3, 0, M, K)).cuda())
+        y = torch.empty((M, N), device="cuda")
+        for _ in range(3):
+            sbm.w4a8_gemm(q, s, nat, sc, N, out=y)
+        times = []
+        for _ in range(5):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sbm.w4a8_gemm(q, s, nat, sc, N, out=y)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / 1e3)
+        t = statistics.median(times)
+        tops = 2.0 * M * N * K / t / 1e12
+        pre[f"K{K}_N{N}"] = {"us": round(t * 1e6, 1), "int_tops": round(tops, 1),
+                             "frac_of_int8_peak": round(tops / int8_peak, 4),
+                             "frac_of_library_int8": round(tops / lib_tops, 4)}
+    out["prefill_M2048"] = pre
+    return out
 
 
 def profile_case(args):
@@ -595,6 +660,20 @@ def profile_case(args):
     import synth
     torch.cuda.set_device(0)
     sbm.load()
+    if args.profile_case == "w4a8":
+        M, K, N = 2048, 4096, 14336
+        w4, scale = sbm.w4a8_pack(synth.config_weights(3, 0, K, N))
+        nat = sbm.w4a8_repack(torch.from_numpy(w4).cuda(), N, K)
+        sc = torch.from_numpy(scale).cuda()
+        q, s = sbm.quant_act(torch.from_numpy(synth.config_activations(3, 0, M, K)).cuda())
+        y = torch.empty((M, N), device="cuda")
+        for _ in range(4):
+            sbm.w4a8_gemm(q, s, nat, sc, N, out=y)
+        torch.cuda.synchronize()
+        status = sbm.last_device_status()
+        print(json.dumps({"profile_case": "w4a8", "M": M, "K": K, "N": N, "launches": 4,
+                          "device_status": status}))
+        return 0 if status == 0 else 1
     M, K, N = (1, 4096, 14336) if args.profile_case == "decode" else (2048, 4096, 14336)
     copies = 8 if M == 1 else 1
     layers = []

@@ -285,6 +285,85 @@ int sherry_gemm_noalloc(const int8_t* x_i8, const float* x_scale, const void* Wn
                         const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,
                         int64_t K, void* stream);
 
+/* ===========================================================================
+ * W4A8 FastGEMM -- the second workload of this library: per-channel SINT4
+ * weights times int8 activations on the same tcgen05 kernel.
+ * (OdysseyLLM review page, xllm-io.github.io/paper-review/blog/odysseyllm,
+ * "OdysseyLLM: A Speed Odyssey for Deployable Quantization of LLMs".)
+ *   - sec. 3.3: symmetric per-channel weight scale
+ *     S[n] = max(|max_k W[n][k]|, |min_k W[n][k]|) / 7, and
+ *     W_q = clamp(rint(W / S), -8, 7) (fp32 IEEE division, ties to even).
+ *     The page's learnable clipping factors are taken as 1.  S = 0 and
+ *     W_q = 0 for an all-zero row.
+ *   - sec. 3.2 / 5.2: SINT4toS8.  The 4-bit two's complement value becomes
+ *     the int8 value 16 w by moving it into the high half of a byte.  An
+ *     int8 GEMM sums q * 16 w exactly in int32.
+ *   - sec. 3.1 (Figure 2, the W4A8 row): those sums are divided by 16
+ *     (exact) before dequantisation:
+ *         acc[m][n] = (sum_k x_i8[m][k] * 16 W_q[n][k]) / 16
+ *         y[m][n]   = (float)((float)acc[m][n] * S[n]) * x_scale[m]
+ * Activations come from sherry_quant_act (per-token absmax / 127).
+ * Canonical SINT4 rows: row n starts at byte n * K/2; byte j holds W_q[n][2j]
+ * in bits 0-3 and W_q[n][2j+1] in bits 4-7 (two's complement nibbles).
+ * Shape rules: those of the Sherry path, and K <= 132104 (so K <= 132096
+ * with K % 32 == 0) so that
+ * |sum q * 16 w| <= 127 * 128 * K stays below 2^31.
+ * =========================================================================== */
+
+/* Bytes of canonical SINT4 rows: N * K/2; 0 when (N, K) is not supported. */
+size_t sherry_w4a8_packed_bytes(int64_t N, int64_t K);
+/* Bytes of the kernel-native SINT4 layout written by sherry_w4a8_repack:
+ * ceil(N/128) * ceil(K/128) * 8192; 0 when (N, K) is not supported. */
+size_t sherry_w4a8_native_bytes(int64_t N, int64_t K);
+
+/*
+ * sherry_w4a8_pack -- host, synchronous.  Quantises W (sec. 3.3 above) and
+ * packs it into canonical SINT4 rows.
+ *   W      [in]  fp32 [N][K], host memory
+ *   w4     [out] sherry_w4a8_packed_bytes(N, K) bytes, host memory
+ *   scale  [out] fp32 [N] per-channel scales S, host memory
+ * Returns SHERRY_ERR_NONFINITE (nothing written) when W holds a NaN or Inf,
+ * SHERRY_ERR_UNSUPPORTED_SHAPE for K % 32 != 0 or K > 132104.
+ */
+int sherry_w4a8_pack(const float* W, int64_t N, int64_t K, uint8_t* w4, float* scale);
+
+/* sherry_w4a8_unpack -- host, synchronous.  Canonical SINT4 rows -> int8
+ * W_q [N][K] with values in [-8, 7] (tests and inspection). */
+int sherry_w4a8_unpack(const uint8_t* w4, int64_t N, int64_t K, int8_t* Wq);
+
+/*
+ * sherry_w4a8_repack -- device, asynchronous on `stream`.  Rearranges
+ * canonical SINT4 rows into the layout sherry_w4a8_gemm reads.  Run it once
+ * per weight matrix; the output does not depend on the GPU.
+ *   w4_dev     [in]  canonical rows, device memory
+ *   native_dev [out] sherry_w4a8_native_bytes(N, K) bytes, device memory,
+ *                    16-byte aligned
+ */
+int sherry_w4a8_repack(const uint8_t* w4_dev, int64_t N, int64_t K, void* native_dev,
+                       void* stream);
+
+/*
+ * sherry_w4a8_gemm_acc -- device, asynchronous.  The W4A8 contraction and
+ * dequantisation above, on the tcgen05 tensor-core kernel for every M: the
+ * SINT4toS8 conversion runs in the kernel's decoder warps, between the
+ * shared-memory copy of the weights and the tensor memory the MMAs read.
+ *   x_i8, x_scale  [in]  from sherry_quant_act, device memory (x_i8 16-byte aligned)
+ *   W4native       [in]  from sherry_w4a8_repack, device memory, 16-byte aligned
+ *   scale          [in]  fp32 [N] per-channel S from sherry_w4a8_pack, device memory
+ *   y              [out] fp32 [M][N] or NULL
+ *   acc            [out] int32 [M][N] (the sums after the division by 16) or NULL
+ * At least one of y and acc must be non-NULL.  Uses the split-K workspace
+ * described at the top of this file.
+ */
+int sherry_w4a8_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* W4native,
+                         const float* scale, float* y, int32_t* acc, int64_t M, int64_t N,
+                         int64_t K, void* stream);
+
+/* sherry_w4a8_gemm -- sherry_w4a8_gemm_acc without the int32 output (y required). */
+int sherry_w4a8_gemm(const int8_t* x_i8, const float* x_scale, const void* W4native,
+                     const float* scale, float* y, int64_t M, int64_t N, int64_t K,
+                     void* stream);
+
 /*
  * sherry_last_device_status -- host, synchronous (copies one word from the
  * current device).  0 when no kernel of this library has reported a bounded

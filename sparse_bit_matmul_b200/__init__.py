@@ -25,6 +25,8 @@ ABI_SYMBOLS = (
     "sherry_pack", "sherry_unpack", "sherry_repack", "sherry_quant_act", "sherry_gemm",
     "sherry_gemm_acc", "sherry_gemm_tc", "sherry_gemm_gemv", "sherry_gemm_simt", "sherry_gemm_noalloc",
     "sherry_gemm_decode", "sherry_linear", "sherry_linear_ex", "sherry_last_device_status",
+    "sherry_w4a8_packed_bytes", "sherry_w4a8_native_bytes", "sherry_w4a8_pack", "sherry_w4a8_unpack",
+    "sherry_w4a8_repack", "sherry_w4a8_gemm", "sherry_w4a8_gemm_acc",
 )
 
 _lib = None
@@ -66,6 +68,15 @@ def load() -> ctypes.CDLL:
     L.sherry_linear.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_linear_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_last_device_status.argtypes = [c_int]
+    L.sherry_w4a8_packed_bytes.argtypes = [i64, i64]
+    L.sherry_w4a8_packed_bytes.restype = ctypes.c_size_t
+    L.sherry_w4a8_native_bytes.argtypes = [i64, i64]
+    L.sherry_w4a8_native_bytes.restype = ctypes.c_size_t
+    L.sherry_w4a8_pack.argtypes = [vp, i64, i64, vp, vp]
+    L.sherry_w4a8_unpack.argtypes = [vp, i64, i64, vp]
+    L.sherry_w4a8_repack.argtypes = [vp, i64, i64, vp, vp]
+    L.sherry_w4a8_gemm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_w4a8_gemm_acc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     for name in ABI_SYMBOLS:
         getattr(L, name).restype = getattr(L, name).restype or c_int
     _lib = L
@@ -238,3 +249,58 @@ class PackedLinear:
 
     def forward(self, x, out=None):
         return linear(x, self.w_native, self.alpha, self.N, out=out)
+
+
+# ------------------------------------------------ W4A8 FastGEMM (SINT4 x int8)
+def w4a8_packed_bytes(N: int, K: int) -> int:
+    return int(load().sherry_w4a8_packed_bytes(N, K))
+
+
+def w4a8_native_bytes(N: int, K: int) -> int:
+    return int(load().sherry_w4a8_native_bytes(N, K))
+
+
+def w4a8_pack(W: np.ndarray):
+    """fp32 W [N][K] -> (canonical SINT4 rows uint8 [N][K/2], per-channel scale fp32 [N])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    w4 = np.empty((N, K // 2), dtype=np.uint8)
+    scale = np.empty(N, dtype=np.float32)
+    _check(load().sherry_w4a8_pack(_np_ptr(W), N, K, _np_ptr(w4), _np_ptr(scale)), "sherry_w4a8_pack")
+    return w4, scale
+
+
+def w4a8_unpack(w4: np.ndarray, K: int) -> np.ndarray:
+    w4 = np.ascontiguousarray(w4, dtype=np.uint8)
+    N = w4.shape[0]
+    Wq = np.empty((N, K), dtype=np.int8)
+    _check(load().sherry_w4a8_unpack(_np_ptr(w4), N, K, _np_ptr(Wq)), "sherry_w4a8_unpack")
+    return Wq
+
+
+def w4a8_repack(w4_dev, N: int, K: int, out=None):
+    """Canonical SINT4 rows on the device -> kernel-native layout (uint8 tensor)."""
+    import torch
+    if out is None:
+        out = torch.empty(w4a8_native_bytes(N, K), dtype=torch.uint8, device=w4_dev.device)
+    _check(load().sherry_w4a8_repack(_dptr(w4_dev), N, K, _dptr(out), _stream(w4_dev)), "sherry_w4a8_repack")
+    return out
+
+
+def w4a8_gemm(x_i8, x_scale, w4_native, scale, N: int, out=None, acc=None, want_y: bool = True):
+    """y fp32 [M][N] (and optionally the int32 sums after the division by 16)
+    from int8 activations and kernel-native SINT4 weights."""
+    import torch
+    M, K = x_i8.shape
+    y = None
+    if want_y:
+        y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x_i8.device)
+    L = load()
+    if acc is None:
+        rc = L.sherry_w4a8_gemm(_dptr(x_i8), _dptr(x_scale), _dptr(w4_native), _dptr(scale), _dptr(y), M, N, K,
+                                _stream(x_i8))
+    else:
+        rc = L.sherry_w4a8_gemm_acc(_dptr(x_i8), _dptr(x_scale), _dptr(w4_native), _dptr(scale), _dptr(y),
+                                    _dptr(acc), M, N, K, _stream(x_i8))
+    _check(rc, "sherry_w4a8_gemm")
+    return y

@@ -340,5 +340,12 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
+// 16-byte shared load (addr 16-byte aligned)
+__device__ __forceinline__ void lds_v4_u32(uint32_t addr, uint32_t (&v)[4])
+{
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(addr));
+}
 }  // namespace ptx
 }  // namespace sherry

@@ -88,6 +88,20 @@ __global__ void repack_kernel(const uint8_t* __restrict__ codes, int64_t N, int6
 }
 
 // ---------------------------------------------------------------------------
+// W4A8 repack: canonical SINT4 rows [N][K/2] (even k in the low nibble) ->
+// the native blocks of sherry_internal.h (one thread per native word).
+// Rows past N and chunks past K are zero.
+// ---------------------------------------------------------------------------
+__global__ void repack_w4_kernel(const uint8_t* __restrict__ w4, int64_t N, int64_t K, uint32_t* __restrict__ out,
+                                 int64_t total_words)
+{
+    const int64_t Kc = sherry_k_chunks(K);
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total_words;
+         idx += (int64_t)gridDim.x * blockDim.x)
+        out[idx] = sherry_w4_native_word(w4, N, K, Kc, idx);
+}
+
+// ---------------------------------------------------------------------------
 // SIMT comparison kernel: thread = weight row, MT tokens per CTA, decode
 // through a 32-entry shared table, dp4a against the activations.
 // ---------------------------------------------------------------------------
@@ -317,11 +331,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <int BN, int SC>
+template <int BN, int SC, int WF = tc::kWeightSherry>
 int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y, int32_t* acc,
               int64_t M, int64_t N, int64_t K, cudaStream_t stream)
 {
-    using C = tc::Cfg<BN, SC>;
+    using C = tc::Cfg<BN, SC, WF>;
     DeviceInfo di;
     int st = device_info(&di);
     if (st != SHERRY_OK) return st;
@@ -359,10 +373,10 @@ int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alp
     // one 512-column tensor-memory allocation) lives on each SM
     const int smem = std::max(C::kSmemBytes, 120 * 1024);
     if (smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
-    cudaError_t e = cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN, SC>,
+    cudaError_t e = cudaFuncSetAttribute(tc::sherry_gemm_tc_kernel<BN, SC, WF>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return SHERRY_ERR_CUDA;
-    e = launch_pdl(tc::sherry_gemm_tc_kernel<BN, SC>, dim3((unsigned)grid), dim3(C::kThreads), (size_t)smem,
+    e = launch_pdl(tc::sherry_gemm_tc_kernel<BN, SC, WF>, dim3((unsigned)grid), dim3(C::kThreads), (size_t)smem,
                    stream, map, ymap, p);
     if (e != cudaSuccess) return cuda_status(e);
     return cuda_status(cudaGetLastError());
@@ -648,6 +662,45 @@ int sherry_repack(const uint8_t* codes_dev, int64_t N, int64_t K, void* native_d
     repack_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
         codes_dev, N, K, static_cast<uint32_t*>(native_dev), words);
     return cuda_status(cudaGetLastError());
+}
+
+int sherry_w4a8_repack(const uint8_t* w4_dev, int64_t N, int64_t K, void* native_dev, void* stream)
+{
+    if (!w4_dev || !native_dev) return SHERRY_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0) return SHERRY_ERR_INVALID_ARG;
+    const size_t bytes = sherry_w4a8_native_bytes(N, K);
+    if (bytes == 0) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(native_dev)) return SHERRY_ERR_INVALID_ARG;
+    const int64_t words = (int64_t)(bytes / 4);
+    const int threads = 256;
+    const int64_t blocks = std::min<int64_t>((words + threads - 1) / threads, 148 * 32);
+    repack_w4_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        w4_dev, N, K, static_cast<uint32_t*>(native_dev), words);
+    return cuda_status(cudaGetLastError());
+}
+
+int sherry_w4a8_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* W4native, const float* scale,
+                         float* y, int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    int st = check_gemm_args(x_i8, x_scale, W4native, scale, y, acc, M, N, K);
+    if (st != SHERRY_OK) return st;
+    if (K > SHERRY_W4_MAX_K) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    constexpr int W4 = tc::kWeightInt4;
+    // int4 stages carry 3.2x the weight bytes of code stages: two-chunk
+    // stages from 32 tokens on keep at least three stages in the ring
+    if (M <= 16) return launch_tc<16, 4, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+    if (M <= 32) return launch_tc<32, 2, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+    if (M <= 64) return launch_tc<64, 2, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+    if (M < 1536) return launch_tc<128, 2, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+    return launch_tc<192, 1, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+}
+
+int sherry_w4a8_gemm(const int8_t* x_i8, const float* x_scale, const void* W4native, const float* scale, float* y,
+                     int64_t M, int64_t N, int64_t K, void* stream)
+{
+    if (!y) return SHERRY_ERR_INVALID_ARG;
+    return sherry_w4a8_gemm_acc(x_i8, x_scale, W4native, scale, y, nullptr, M, N, K, stream);
 }
 
 int sherry_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_i8, float* x_scale, void* stream)

@@ -148,4 +148,78 @@ int sherry_unpack(const uint8_t* codes, int64_t N, int64_t K, int8_t* T)
     return SHERRY_OK;
 }
 
+// ---------------------------------------------------------------------------
+// W4A8 FastGEMM weights (OdysseyLLM review page,
+// xllm-io.github.io/paper-review/blog/odysseyllm, sec. 3.3 and 5.2): one
+// symmetric scale per output channel, S = a / 7 with a the largest |w| of
+// the row (the clipping factors taken as 1), w_q = clamp(rint(w / S), -8, 7)
+// in fp32 (IEEE division, ties to even); a == 0 gives S = 0 and w_q = 0.
+// Stored as 4-bit two's complement, two per byte, even k in the low nibble.
+// ---------------------------------------------------------------------------
+
+static bool w4a8_shape_ok(int64_t M, int64_t N, int64_t K)
+{
+    return sherry_shape_ok(M, N, K) && K <= SHERRY_W4_MAX_K;
+}
+
+size_t sherry_w4a8_packed_bytes(int64_t N, int64_t K)
+{
+    if (!w4a8_shape_ok(1, N, K)) return 0;
+    return (size_t)N * (size_t)(K / 2);
+}
+
+size_t sherry_w4a8_native_bytes(int64_t N, int64_t K)
+{
+    if (!w4a8_shape_ok(1, N, K)) return 0;
+    return (size_t)sherry_row_tiles(N) * (size_t)sherry_k_chunks(K) * SHERRY_W4_CHUNK_BYTES;
+}
+
+int sherry_w4a8_pack(const float* W, int64_t N, int64_t K, uint8_t* w4, float* scale)
+{
+    if (!W || !w4 || !scale) return SHERRY_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0) return SHERRY_ERR_INVALID_ARG;
+    if (!w4a8_shape_ok(1, N, K)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    int nonfinite = 0;
+#pragma omp parallel for schedule(static) reduction(| : nonfinite)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) nonfinite |= ((float_bits(W[n * K + k]) & 0x7f800000u) == 0x7f800000u);
+    if (nonfinite) return SHERRY_ERR_NONFINITE;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const float* w = W + n * K;
+        uint8_t* out = w4 + n * (K / 2);
+        float a = 0.0f;
+        for (int64_t k = 0; k < K; ++k) a = std::fmax(a, std::fabs(w[k]));
+        const float S = a / 7.0f;
+        scale[n] = S;
+        for (int64_t k = 0; k < K; k += 2) {
+            uint32_t nib[2] = {0u, 0u};
+            if (a != 0.0f) {
+                for (int e = 0; e < 2; ++e) {
+                    const float r = std::fmin(std::fmax(std::rint(w[k + e] / S), -8.0f), 7.0f);
+                    nib[e] = (uint32_t)(int32_t)r & 0xFu;
+                }
+            }
+            out[k / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
+        }
+    }
+    return SHERRY_OK;
+}
+
+int sherry_w4a8_unpack(const uint8_t* w4, int64_t N, int64_t K, int8_t* Wq)
+{
+    if (!w4 || !Wq) return SHERRY_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0) return SHERRY_ERR_INVALID_ARG;
+    if (!w4a8_shape_ok(1, N, K)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K / 2; ++j) {
+            const uint8_t b = w4[n * (K / 2) + j];
+            // sign-extend each nibble: (v ^ 8) - 8
+            Wq[n * K + 2 * j] = (int8_t)((int)((b & 0xFu) ^ 8u) - 8);
+            Wq[n * K + 2 * j + 1] = (int8_t)((int)((b >> 4) ^ 8u) - 8);
+        }
+    return SHERRY_OK;
+}
+
 }  // extern "C"

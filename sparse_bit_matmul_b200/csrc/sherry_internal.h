@@ -19,6 +19,17 @@
 #define SHERRY_CHUNK_WORDS 5
 #define SHERRY_CHUNK_BYTES_PER_TILE (SHERRY_TILE_ROWS * SHERRY_CHUNK_WORDS * 4)
 
+// W4A8 (SINT4 weights) kernel-native layout: the same row tiles and K chunks;
+// one (tile, chunk) block is 8192 bytes, [piece q 0..3][row r 0..127][word i
+// 0..3] of 32-bit words.  Word i of piece q of row r covers k0 = 32q + 8i
+// within the chunk: byte b holds w[k0 + b] in its low nibble and w[k0 + 4 + b]
+// in its high nibble.  So (word << 4) & 0xF0F0F0F0 and word & 0xF0F0F0F0 are
+// the int8 values 16 w of k0..k0+3 and k0+4..k0+7, and a warp loading the
+// 16-byte pieces of 32 consecutive rows reads 512 contiguous bytes.
+#define SHERRY_W4_CHUNK_BYTES (SHERRY_TILE_ROWS * SHERRY_KCHUNK / 2)
+// Largest K of the W4A8 path: |sum of q * 16 w| <= 127 * 128 * K below 2^31.
+#define SHERRY_W4_MAX_K int64_t(132104)
+
 // Largest supported K: keeps |acc| <= 127 * 0.75 * K below 2^31.
 #define SHERRY_MAX_K (int64_t(1) << 24)
 #define SHERRY_MAX_DIM ((int64_t(1) << 31) - 1)
@@ -41,6 +52,30 @@ SHERRY_HD inline int64_t sherry_k_chunks(int64_t K) { return (K + SHERRY_KCHUNK 
 SHERRY_HD inline int sherry_word_pos(int j, int r)
 {
     return j * SHERRY_TILE_ROWS + ((r + 8 * j) & (SHERRY_TILE_ROWS - 1));
+}
+
+// Word index of (piece q, row r, word i) inside one W4A8 (tile, chunk) block.
+SHERRY_HD inline int sherry_w4_word_index(int q, int r, int i) { return (q * SHERRY_TILE_ROWS + r) * 4 + i; }
+
+// Native W4A8 word `idx` built from canonical SINT4 rows w4 [N][K/2] (even k
+// in the low nibble), K % 32 == 0, Kc = K chunks.  Rows past N and chunks
+// past K give 0.
+SHERRY_HD inline uint32_t sherry_w4_native_word(const uint8_t* w4, int64_t N, int64_t K, int64_t Kc, int64_t idx)
+{
+    const int i = (int)(idx & 3);
+    const int r = (int)((idx >> 2) & (SHERRY_TILE_ROWS - 1));
+    const int q = (int)((idx >> 9) & 3);
+    const int64_t blk = idx >> 11;                         // (tile, chunk) block of 2048 words
+    const int64_t c = blk % Kc, t = blk / Kc;
+    const int64_t n = t * SHERRY_TILE_ROWS + r;
+    const int64_t k0 = c * SHERRY_KCHUNK + 32 * q + 8 * i;
+    if (n >= N || k0 >= K) return 0u;                      // K % 32 == 0: all 8 weights are in range
+    const uint8_t* src = w4 + n * (K / 2) + k0 / 2;
+    uint32_t u = 0;                                        // nibble e = w[k0 + e]
+    for (int b = 0; b < 4; ++b) u |= (uint32_t)src[b] << (8 * b);
+    uint32_t w = 0;
+    for (int b = 0; b < 4; ++b) w |= (((u >> (4 * b)) & 0xFu) | (((u >> (16 + 4 * b)) & 0xFu) << 4)) << (8 * b);
+    return w;
 }
 
 // Codes reported through sherry_last_device_status when a bounded wait runs out.

@@ -45,6 +45,15 @@
 // Every wait is bounded in wall time; when a bound runs out the kernel
 // records a status code, stops issuing work, waits (bounded) for what it has
 // in flight, frees its tensor memory and returns.
+//
+// The same kernel runs the W4A8 FastGEMM of the OdysseyLLM review page
+// (xllm-io.github.io/paper-review/blog/odysseyllm, sec. 3.1-3.2, 5.2) when
+// WF = kWeightInt4: the weights are per-channel SINT4 (8 KB per 128 x 128
+// chunk instead of 2560 bytes of codes), the decoders turn each 4-bit two's
+// complement value into the int8 16 w by moving it into the high half of a
+// byte (shift and mask, no table), the MMAs sum q * 16 w exactly in int32,
+// and the epilogue divides those sums by 16 (an exact arithmetic shift)
+// before the two fp32 products with the channel scale and the token scale.
 #pragma once
 
 #include <cstdint>
@@ -60,10 +69,13 @@ constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kDecWarp0 = 2;
 constexpr int kTmemCols = 512;
-constexpr int kChunkCodeBytes = SHERRY_CHUNK_BYTES_PER_TILE;   // 2560
 constexpr uint64_t kWaitLimitNs = 2000000000ull;              // 2 s per wait
 
-template <int BN, int SC>
+// weight formats
+constexpr int kWeightSherry = 0;     // 5-bit 3:4 ternary group codes
+constexpr int kWeightInt4 = 1;       // SINT4, two per byte
+
+template <int BN, int SC, int WF = kWeightSherry>
 struct Cfg {
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 192, "BN");
     // 192-token tiles: two 192-column accumulators leave 128 TMEM columns:
@@ -74,11 +86,18 @@ struct Cfg {
     static constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;
     static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
     static_assert(SC >= 1 && SC <= 4, "SC");
+    static_assert(WF == kWeightSherry || WF == kWeightInt4, "WF");
+    // weight bytes of one (row tile, K chunk) block
+    static constexpr int kChunkWBytes = WF == kWeightSherry ? SHERRY_CHUNK_BYTES_PER_TILE : SHERRY_W4_CHUNK_BYTES;
+    // int32 sums of q * 16 w are divided by 16 before the epilogue uses them
+    static constexpr int kAccShift = WF == kWeightInt4 ? 4 : 0;
     static constexpr int kBChunkBytes = BN * 128;
     static constexpr int kBStageBytes = SC * kBChunkBytes;
-    static constexpr int kCodeStageBytes = SC * kChunkCodeBytes;
+    static constexpr int kCodeStageBytes = SC * kChunkWBytes;
     static constexpr int kStageBytes = kBStageBytes + kCodeStageBytes;
-    static constexpr int kStagesRaw = (192 * 1024) / kStageBytes;
+    // the int4 stages leave 4 KB of the 192 KB ring budget for the larger
+    // fixed part (barriers, scales, store staging, the table's static array)
+    static constexpr int kStagesRaw = (192 * 1024 - (WF == kWeightInt4 ? 4096 : 0)) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static constexpr int kACols = 32 * SC;                          // TMEM columns of one A stage
     static constexpr int kDBufs = (2 * BN + 2 * kACols <= kTmemCols) ? 2 : 1;
@@ -101,6 +120,9 @@ struct Cfg {
     static constexpr int kOffStaging = (kOffMisc + kMiscBytes + 127) & ~127;
     static constexpr int kStagingBytes = 4 * 2 * kSlice * 32 * 4;
     static constexpr int kSmemBytes = kOffStaging + kStagingBytes + 1024;   // + alignment slack
+    // dynamic plus static (the table of the code path, 1 KB as compiled)
+    // within the 227 KB per-block limit
+    static_assert(kSmemBytes + (WF == kWeightSherry ? 1024 : 0) <= 232448, "shared memory");
     // instruction descriptor: s32 accumulate, signed int8 A and B, both
     // K-major, N = BN, M = 128
     static constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
@@ -257,12 +279,12 @@ struct StageWalk {
     }
 };
 
-template <int BN, int SC>
-__global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
+template <int BN, int SC, int WF = kWeightSherry>
+__global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
     sherry_gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap,
                           const Params p)
 {
-    using C = Cfg<BN, SC>;
+    using C = Cfg<BN, SC, WF>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ __align__(128) uint32_t table[32];
     // 1024-byte aligned start, computed by pointer arithmetic so that the
@@ -286,7 +308,7 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
 
     const int64_t G = gridDim.x;
 
-    if (threadIdx.x < 32) {
+    if (WF == kWeightSherry && threadIdx.x < 32) {
         // code -> four int8 weights of the group, byte i = position i
         const uint32_t c = threadIdx.x, z = c & 3u;
         uint32_t word = 0, slot = 2;
@@ -350,7 +372,7 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
         while (!w.done()) {
             const int64_t tm = w.tile / p.TN, tn = w.tile - tm * p.TN;
             int c = (int)w.cb;                     // K chunk within the tile
-            const uint8_t* src = p.wnative + (tn * p.Kc + c) * (int64_t)kChunkCodeBytes;
+            const uint8_t* src = p.wnative + (tn * p.Kc + c) * (int64_t)C::kChunkWBytes;
             const int32_t ty = (int32_t)(tm * BN);
             int left = (int)(w.ce - w.cb);
             while (left > 0) {
@@ -362,9 +384,9 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
                 const int s1 = (s + 1 == C::kStages) ? 0 : s + 1;
                 const uint32_t ph1 = (s + 1 == C::kStages) ? ph ^ 1u : ph;
                 const uint32_t t_e = ptx::mbar_test(empty_bar(s1), ph1 ^ 1u);
-                ptx::mbar_arrive_expect_tx_elect(full_bar(s), (uint32_t)(nch * (kChunkCodeBytes + C::kBChunkBytes)));
+                ptx::mbar_arrive_expect_tx_elect(full_bar(s), (uint32_t)(nch * (C::kChunkWBytes + C::kBChunkBytes)));
                 ptx::bulk_g2s_elect(sbase + C::kOffCodes + (uint32_t)s * C::kCodeStageBytes, src,
-                                    (uint32_t)(nch * kChunkCodeBytes), full_bar(s));
+                                    (uint32_t)(nch * C::kChunkWBytes), full_bar(s));
                 if (nch == SC) {
 #pragma unroll
                     for (int j = 0; j < SC; ++j)
@@ -375,7 +397,7 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
                         ptx::tma_load_2d_elect(sbase + (uint32_t)(s * C::kBStageBytes + j * C::kBChunkBytes), &xmap,
                                                (c + j) * SHERRY_KCHUNK, ty, full_bar(s));
                 }
-                src += nch * kChunkCodeBytes;
+                src += nch * C::kChunkWBytes;
                 c += nch;
                 left -= nch;
                 ++issued;
@@ -504,12 +526,47 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
                     break;
                 }
                 const uint32_t codes_s = sbase + (uint32_t)(C::kOffCodes + s * C::kCodeStageBytes);
+                if constexpr (WF == kWeightInt4) {
+                    // SINT4 -> int8 16 w (shift into the high half of each
+                    // byte); the stage's weights are read while its A slot is
+                    // filled, then both are released
+                    ok = ptx::mbar_wait_bounded(aempty_bar(a), aph ^ 1u, kWaitLimitNs);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
+                        quit = true;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t wrow = codes_s + (uint32_t)(16 * row);
+#pragma unroll
+                    for (int j = 0; j < SC; ++j) {
+                        if (j >= nch) break;
+                        uint32_t a_vals[32];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t v[4];
+                            ptx::lds_v4_u32(wrow + (uint32_t)(j * C::kChunkWBytes + q * SHERRY_TILE_ROWS * 16), v);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                a_vals[8 * q + 2 * i] = (v[i] << 4) & 0xF0F0F0F0u;
+                                a_vals[8 * q + 2 * i + 1] = v[i] & 0xF0F0F0F0u;
+                            }
+                        }
+                        ptx::tmem_st_32x32b_x32(lane_base + (uint32_t)(C::kACol0 + a * C::kACols + 32 * j), a_vals);
+                    }
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(empty_bar(s));
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(afull_bar(a));
+                } else {
                 uint32_t w[SC][SHERRY_CHUNK_WORDS];
 #pragma unroll
                 for (int j = 0; j < SC; ++j)
 #pragma unroll
                     for (int k = 0; k < SHERRY_CHUNK_WORDS; ++k)
-                        w[j][k] = (j < nch) ? ptx::lds_u32(codes_s + (uint32_t)(j * kChunkCodeBytes) + wpos[k]) : 0u;
+                        w[j][k] = (j < nch) ? ptx::lds_u32(codes_s + (uint32_t)(j * C::kChunkWBytes) + wpos[k]) : 0u;
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(empty_bar(s));
                 ok = ptx::mbar_wait_bounded(aempty_bar(a), aph ^ 1u, kWaitLimitNs);
@@ -540,6 +597,7 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(afull_bar(a));
+                }
             }
             if (++s == C::kStages) { s = 0; sph ^= 1u; }
             if (++a == C::kAStages) { a = 0; aph ^= 1u; }
@@ -608,7 +666,8 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
                     float* stg = stg_w + (stage_slice & 1) * (SL * 32);
 #pragma unroll
                     for (int jj = 0; jj < SL; ++jj)
-                        stg[jj * 32 + lane] = __fmul_rn(__fmul_rn((float)(int32_t)v[jj], al), sc_s[j0 + jj]);
+                        stg[jj * 32 + lane] =
+                            __fmul_rn(__fmul_rn((float)((int32_t)v[jj] >> C::kAccShift), al), sc_s[j0 + jj]);
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
@@ -628,11 +687,12 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
                 for (int jj = 0; jj < 16; ++jj) {
                     const int64_t m = tm * BN + j0 + jj;
                     if (m >= p.M) continue;
-                    const int32_t a32 = (int32_t)v[jj];
+                    const int32_t a32 = (int32_t)v[jj];      // a partial sum goes to the slot as is
                     if (complete) {
+                        const int32_t af = a32 >> C::kAccShift;
                         if (n < p.N) {
-                            if (p.acc) p.acc[m * p.N + n] = a32;
-                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, al), sc_s[j0 + jj]);
+                            if (p.acc) p.acc[m * p.N + n] = af;
+                            if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)af, al), sc_s[j0 + jj]);
                         }
                     } else {
                         ptx::red_add_s32(wsl + (j0 + jj) * SHERRY_TILE_ROWS + r, a32);
@@ -671,9 +731,10 @@ __global__ void __launch_bounds__(Cfg<BN, SC>::kThreads, 1)
                             if (j >= jn) break;
                             const int64_t m = cur_tm * BN + j;
                             wsl[j * SHERRY_TILE_ROWS + r] = 0;
+                            const int32_t af = v[jj] >> C::kAccShift;
                             if (n < p.N) {
-                                if (p.acc) p.acc[m * p.N + n] = v[jj];
-                                if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)v[jj], al), sc_s[j]);
+                                if (p.acc) p.acc[m * p.N + n] = af;
+                                if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)af, al), sc_s[j]);
                             }
                         }
                     }
