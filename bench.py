@@ -55,8 +55,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "w4a8"], default=None,
-                    help="run a few launches of one layer shape (K=4096, N=14336; M=1 or 2048; "
+    ap.add_argument("--profile-case", choices=["decode", "small", "prefill", "w4a8"], default=None,
+                    help="run a few launches of one layer shape (K=4096, N=14336; M=1, 16 or 2048; "
                          "w4a8: the SINT4 x int8 GEMM at M=2048) and exit: the target of the "
                          "committed ncu captures")
     return ap.parse_args(argv)
@@ -674,13 +674,14 @@ def profile_case(args):
         print(json.dumps({"profile_case": "w4a8", "M": M, "K": K, "N": N, "launches": 4,
                           "device_status": status}))
         return 0 if status == 0 else 1
-    M, K, N = (1, 4096, 14336) if args.profile_case == "decode" else (2048, 4096, 14336)
-    copies = 8 if M == 1 else 1
+    M = {"decode": 1, "small": 16, "prefill": 2048}[args.profile_case]
+    K, N = 4096, 14336
+    copies = 8 if M <= 16 else 1
     layers = []
     for c in range(copies):
-        codes, alpha = sbm.pack(synth.config_weights(1 if M == 1 else 3, c, K, N))
+        codes, alpha = sbm.pack(synth.config_weights(1 if M <= 16 else 3, c, K, N))
         layers.append((sbm.repack(torch.from_numpy(codes).cuda(), N, K), torch.from_numpy(alpha).cuda()))
-    x = torch.from_numpy(synth.config_activations(1 if M == 1 else 3, 0, M, K)).cuda()
+    x = torch.from_numpy(synth.config_activations(1 if M == 1 else (2 if M <= 16 else 3), 0, M, K)).cuda()
     q, s = sbm.quant_act(x)
     y = torch.empty((M, N), device="cuda")
     kernel = "auto" if args.impl == "reference" else args.impl
