@@ -602,7 +602,8 @@ def w4a8_extras(args, flush, int8_peak, lib_tops, world):
     import torch
     import sparse_bit_matmul_b200 as sbm
     import synth
-    out = {"kernel": "sherry_gemm_tc_kernel<BN, SC, int4 weights> via sherry_w4a8_gemm",
+    out = {"kernel": "sherry_w4a8_gemm: w4a8_gemv_kernel (CUDA cores) for M <= 4, "
+                     "sherry_gemm_tc_kernel<BN, SC, int4 weights> above",
            "weights": "synthetic N(0, 0.02) quantised per channel to SINT4 (S = max|w| / 7)"}
     K, N = 4096, 14336
     copies = 9                                    # 9 x 29.4 MB = 264 MB > 2 x L2
@@ -611,7 +612,7 @@ def w4a8_extras(args, flush, int8_peak, lib_tops, world):
         w4, scale = sbm.w4a8_pack(synth.config_weights(1, c, K, N))
         mats.append((sbm.w4a8_repack(torch.from_numpy(w4).cuda(), N, K), torch.from_numpy(scale).cuda()))
     small = {}
-    for M in (1, 16):
+    for M in (1, 4, 16):
         q, s = sbm.quant_act(torch.from_numpy(synth.config_activations(2, 0, M, K)).cuda())
         y = torch.empty((M, N), device="cuda")
 

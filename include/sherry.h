@@ -342,22 +342,45 @@ int sherry_w4a8_unpack(const uint8_t* w4, int64_t N, int64_t K, int8_t* Wq);
 int sherry_w4a8_repack(const uint8_t* w4_dev, int64_t N, int64_t K, void* native_dev,
                        void* stream);
 
+/* Largest M that sherry_w4a8_gemm sends to the CUDA-core GEMV. */
+#define SHERRY_W4A8_GEMV_MAX_M 4
+
 /*
  * sherry_w4a8_gemm_acc -- device, asynchronous.  The W4A8 contraction and
- * dequantisation above, on the tcgen05 tensor-core kernel for every M: the
- * SINT4toS8 conversion runs in the kernel's decoder warps, between the
- * shared-memory copy of the weights and the tensor memory the MMAs read.
+ * dequantisation above.  M <= SHERRY_W4A8_GEMV_MAX_M runs
+ * sherry_w4a8_gemm_gemv; larger M runs sherry_w4a8_gemm_tc.
  *   x_i8, x_scale  [in]  from sherry_quant_act, device memory (x_i8 16-byte aligned)
  *   W4native       [in]  from sherry_w4a8_repack, device memory, 16-byte aligned
  *   scale          [in]  fp32 [N] per-channel S from sherry_w4a8_pack, device memory
  *   y              [out] fp32 [M][N] or NULL
  *   acc            [out] int32 [M][N] (the sums after the division by 16) or NULL
- * At least one of y and acc must be non-NULL.  Uses the split-K workspace
- * described at the top of this file.
+ * At least one of y and acc must be non-NULL.  The tensor-core kernel uses
+ * the split-K workspace described at the top of this file.
  */
 int sherry_w4a8_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* W4native,
                          const float* scale, float* y, int32_t* acc, int64_t M, int64_t N,
                          int64_t K, void* stream);
+
+/*
+ * sherry_w4a8_gemm_tc -- device, asynchronous.  The same, on the tcgen05
+ * tensor-core kernel for every M.  The SINT4toS8 conversion runs in the
+ * kernel's decoder warps, between the shared-memory copy of the weights and
+ * the tensor memory the MMAs read.  Arguments as sherry_w4a8_gemm_acc.
+ */
+int sherry_w4a8_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* W4native,
+                        const float* scale, float* y, int32_t* acc, int64_t M, int64_t N,
+                        int64_t K, void* stream);
+
+/*
+ * sherry_w4a8_gemm_gemv -- device, asynchronous.  The same, for M <=
+ * SHERRY_W4A8_GEMV_MAX_M, on the CUDA cores.  A CTA owns 32 rows and splits
+ * K among its warps; the shift into int8 and dp4a run in registers.  Larger
+ * M returns SHERRY_ERR_UNSUPPORTED_SHAPE.  Needs no workspace.  Arguments as
+ * sherry_w4a8_gemm_acc.
+ */
+int sherry_w4a8_gemm_gemv(const int8_t* x_i8, const float* x_scale, const void* W4native,
+                          const float* scale, float* y, int32_t* acc, int64_t M, int64_t N,
+                          int64_t K, void* stream);
 
 /* sherry_w4a8_gemm -- sherry_w4a8_gemm_acc without the int32 output (y required). */
 int sherry_w4a8_gemm(const int8_t* x_i8, const float* x_scale, const void* W4native,

@@ -26,7 +26,8 @@ ABI_SYMBOLS = (
     "sherry_gemm_acc", "sherry_gemm_tc", "sherry_gemm_gemv", "sherry_gemm_simt", "sherry_gemm_noalloc",
     "sherry_gemm_decode", "sherry_linear", "sherry_linear_ex", "sherry_last_device_status",
     "sherry_w4a8_packed_bytes", "sherry_w4a8_native_bytes", "sherry_w4a8_pack", "sherry_w4a8_unpack",
-    "sherry_w4a8_repack", "sherry_w4a8_gemm", "sherry_w4a8_gemm_acc",
+    "sherry_w4a8_repack", "sherry_w4a8_gemm", "sherry_w4a8_gemm_acc", "sherry_w4a8_gemm_tc",
+    "sherry_w4a8_gemm_gemv",
 )
 
 _lib = None
@@ -77,6 +78,8 @@ def load() -> ctypes.CDLL:
     L.sherry_w4a8_repack.argtypes = [vp, i64, i64, vp, vp]
     L.sherry_w4a8_gemm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_w4a8_gemm_acc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_w4a8_gemm_tc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.sherry_w4a8_gemm_gemv.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     for name in ABI_SYMBOLS:
         getattr(L, name).restype = getattr(L, name).restype or c_int
     _lib = L
@@ -287,20 +290,32 @@ def w4a8_repack(w4_dev, N: int, K: int, out=None):
     return out
 
 
-def w4a8_gemm(x_i8, x_scale, w4_native, scale, N: int, out=None, acc=None, want_y: bool = True):
+W4A8_GEMV_MAX_M = 4   # SHERRY_W4A8_GEMV_MAX_M
+
+
+def w4a8_gemm(x_i8, x_scale, w4_native, scale, N: int, out=None, acc=None, want_y: bool = True,
+              kernel: str = "auto"):
     """y fp32 [M][N] (and optionally the int32 sums after the division by 16)
-    from int8 activations and kernel-native SINT4 weights."""
+    from int8 activations and kernel-native SINT4 weights.  kernel: "auto"
+    (the CUDA-core GEMV for M <= 4, tensor cores above), "tc" or "gemv"."""
     import torch
     M, K = x_i8.shape
     y = None
     if want_y:
         y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x_i8.device)
     L = load()
-    if acc is None:
-        rc = L.sherry_w4a8_gemm(_dptr(x_i8), _dptr(x_scale), _dptr(w4_native), _dptr(scale), _dptr(y), M, N, K,
-                                _stream(x_i8))
+    args = (_dptr(x_i8), _dptr(x_scale), _dptr(w4_native), _dptr(scale), _dptr(y), _dptr(acc), M, N, K,
+            _stream(x_i8))
+    if kernel == "auto":
+        if acc is None:
+            rc = L.sherry_w4a8_gemm(args[0], args[1], args[2], args[3], args[4], M, N, K, args[-1])
+        else:
+            rc = L.sherry_w4a8_gemm_acc(*args)
+    elif kernel == "tc":
+        rc = L.sherry_w4a8_gemm_tc(*args)
+    elif kernel == "gemv":
+        rc = L.sherry_w4a8_gemm_gemv(*args)
     else:
-        rc = L.sherry_w4a8_gemm_acc(_dptr(x_i8), _dptr(x_scale), _dptr(w4_native), _dptr(scale), _dptr(y),
-                                    _dptr(acc), M, N, K, _stream(x_i8))
-    _check(rc, "sherry_w4a8_gemm")
+        raise ValueError(kernel)
+    _check(rc, f"sherry_w4a8_gemm[{kernel}]")
     return y

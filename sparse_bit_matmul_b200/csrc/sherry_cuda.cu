@@ -17,6 +17,7 @@
 #include "decode.cuh"
 #include "quant.cuh"
 #include "tc_gemm.cuh"
+#include "w4a8_gemv.cuh"
 
 namespace sherry {
 
@@ -383,6 +384,29 @@ int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alp
 }
 
 
+// W4A8 GEMV for M <= MT tokens: 32 rows per CTA; 16 K parts (512 threads)
+// when there are at least two CTAs per SM, else 32 (1024 threads) so that
+// each SM keeps enough 16-byte loads in flight.
+template <int MT>
+int launch_w4_gemv(const int8_t* x, const float* xs, const void* wn, const float* scale, float* y, int32_t* acc,
+                   int64_t M, int64_t N, int64_t K, cudaStream_t stream)
+{
+    DeviceInfo di;
+    const int st = device_info(&di);
+    if (st != SHERRY_OK) return st;
+    const int64_t ctas = (N + w4gemv::kRows - 1) / w4gemv::kRows;
+    const uint8_t* w = static_cast<const uint8_t*>(wn);
+    cudaError_t e;
+    if (ctas >= 2 * (int64_t)di.sms)
+        e = launch_pdl(w4gemv::w4a8_gemv_kernel<MT, 16>, dim3((unsigned)ctas), dim3(w4gemv::kRows * 16), 0, stream,
+                       x, xs, w, scale, y, acc, M, N, K);
+    else
+        e = launch_pdl(w4gemv::w4a8_gemv_kernel<MT, 32>, dim3((unsigned)ctas), dim3(w4gemv::kRows * 32), 0, stream,
+                       x, xs, w, scale, y, acc, M, N, K);
+    if (e != cudaSuccess) return cuda_status(e);
+    return cuda_status(cudaGetLastError());
+}
+
 template <int MT>
 int launch_gemv(const int8_t* x, const float* xs, const void* wn, const float* alpha, float* y, int32_t* acc,
                 int64_t M, int64_t N, int64_t K, cudaStream_t stream)
@@ -679,8 +703,20 @@ int sherry_w4a8_repack(const uint8_t* w4_dev, int64_t N, int64_t K, void* native
     return cuda_status(cudaGetLastError());
 }
 
-int sherry_w4a8_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* W4native, const float* scale,
-                         float* y, int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+int sherry_w4a8_gemm_gemv(const int8_t* x_i8, const float* x_scale, const void* W4native, const float* scale,
+                          float* y, int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    int st = check_gemm_args(x_i8, x_scale, W4native, scale, y, acc, M, N, K);
+    if (st != SHERRY_OK) return st;
+    if (K > SHERRY_W4_MAX_K || M > SHERRY_W4A8_GEMV_MAX_M) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 1) return launch_w4_gemv<1>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+    if (M == 2) return launch_w4_gemv<2>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+    return launch_w4_gemv<4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+}
+
+int sherry_w4a8_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* W4native, const float* scale,
+                        float* y, int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
 {
     int st = check_gemm_args(x_i8, x_scale, W4native, scale, y, acc, M, N, K);
     if (st != SHERRY_OK) return st;
@@ -694,6 +730,14 @@ int sherry_w4a8_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* W
     if (M <= 64) return launch_tc<64, 2, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
     if (M < 1536) return launch_tc<128, 2, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
     return launch_tc<192, 1, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
+}
+
+int sherry_w4a8_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* W4native, const float* scale,
+                         float* y, int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
+{
+    if (M >= 1 && M <= SHERRY_W4A8_GEMV_MAX_M)
+        return sherry_w4a8_gemm_gemv(x_i8, x_scale, W4native, scale, y, acc, M, N, K, stream);
+    return sherry_w4a8_gemm_tc(x_i8, x_scale, W4native, scale, y, acc, M, N, K, stream);
 }
 
 int sherry_w4a8_gemm(const int8_t* x_i8, const float* x_scale, const void* W4native, const float* scale, float* y,

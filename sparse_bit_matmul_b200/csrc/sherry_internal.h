@@ -57,6 +57,14 @@ SHERRY_HD inline int sherry_word_pos(int j, int r)
 // Word index of (piece q, row r, word i) inside one W4A8 (tile, chunk) block.
 SHERRY_HD inline int sherry_w4_word_index(int q, int r, int i) { return (q * SHERRY_TILE_ROWS + r) * 4 + i; }
 
+// Byte offset of the 16-byte piece p (k = 32p .. 32p+31) of row n in the
+// native W4A8 layout: chunk c = p / 4, piece q = p % 4 of that chunk.
+SHERRY_HD inline int64_t sherry_w4_piece_offset(int64_t n, int64_t Kc, int64_t p)
+{
+    const int64_t t = n / SHERRY_TILE_ROWS, r = n % SHERRY_TILE_ROWS;
+    return (t * Kc + (p >> 2)) * SHERRY_W4_CHUNK_BYTES + (p & 3) * (SHERRY_TILE_ROWS * 16) + 16 * r;
+}
+
 // Native W4A8 word `idx` built from canonical SINT4 rows w4 [N][K/2] (even k
 // in the low nibble), K % 32 == 0, Kc = K chunks.  Rows past N and chunks
 // past K give 0.

@@ -95,18 +95,30 @@ struct Cfg {
     static constexpr int kBStageBytes = SC * kBChunkBytes;
     static constexpr int kCodeStageBytes = SC * kChunkWBytes;
     static constexpr int kStageBytes = kBStageBytes + kCodeStageBytes;
-    // the int4 stages leave 4 KB of the 192 KB ring budget for the larger
-    // fixed part (barriers, scales, store staging, the table's static array)
-    static constexpr int kStagesRaw = (192 * 1024 - (WF == kWeightInt4 ? 4096 : 0)) / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kStagesRaw = (192 * 1024) / kStageBytes;
+    static constexpr int kStagesCap = kStagesRaw > 12 ? 12 : kStagesRaw;
+    // A whole number of rounds of decoder groups: stage s is then always
+    // decoded by group s mod kDecGroups (see the ring rules below).
+    static constexpr int kStages = kStagesCap - kStagesCap % kDecGroups;
     static constexpr int kACols = 32 * SC;                          // TMEM columns of one A stage
     static constexpr int kDBufs = (2 * BN + 2 * kACols <= kTmemCols) ? 2 : 1;
     static constexpr int kAStagesRaw = (kTmemCols - kDBufs * BN) / kACols;
     static constexpr int kAStages = kAStagesRaw > 8 ? 8 : kAStagesRaw;
-    // A decoder group takes every kDecGroups-th stage.  Its phase-parity waits
-    // are exact only while the barrier it waits on is at most one phase
-    // behind: that holds when both rings are at least kDecGroups deep.
-    static_assert(kStages >= kDecGroups && kAStages >= kDecGroups, "pipeline rings shallower than decoder groups");
+    // A decoder group takes every kDecGroups-th stage.  A parity wait is exact
+    // only while the waiter is not a whole phase ahead of the barrier: a wait
+    // for phase k on a barrier still in phase k-1 sees the parity of phase
+    // k-2, complete, and returns at once.
+    //  - full(s): the copies of different stages may land in any order, so
+    //    the group waiting for the fill of iteration i must itself have seen
+    //    the fill of iteration i - kStages: kStages a multiple of kDecGroups
+    //    makes it the same group.  It cannot be two phases behind either: the
+    //    next refill of stage s needs this group's arrival on empty(s).
+    //  - aempty(a): completed by tcgen05.commit of the one MMA thread, in
+    //    issue order; a group that saw its previous slot freed has seen every
+    //    earlier MMA complete, which covers slot a's previous use once the
+    //    ring is at least kDecGroups deep.
+    static_assert(kStages >= kDecGroups && kStages % kDecGroups == 0, "stage ring not whole rounds of decoder groups");
+    static_assert(kAStages >= kDecGroups, "A ring shallower than decoder groups");
     static constexpr int kACol0 = kDBufs * BN;
     // shared memory: [B stages][code stages][barriers + misc]
     static constexpr int kOffCodes = kStages * kBStageBytes;

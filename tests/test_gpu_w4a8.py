@@ -39,12 +39,12 @@ def upload_w4(W: np.ndarray):
     return native, torch.from_numpy(scale).cuda(), w4, scale
 
 
-def run_w4(x: np.ndarray, native, scale_d, N: int, with_acc: bool = True):
+def run_w4(x: np.ndarray, native, scale_d, N: int, with_acc: bool = True, kernel: str = "auto"):
     xd = torch.from_numpy(np.ascontiguousarray(x)).cuda()
     M = x.shape[0]
     q, s = sbm.quant_act(xd)
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda") if with_acc else None
-    y = sbm.w4a8_gemm(q, s, native, scale_d, N, acc=acc)
+    y = sbm.w4a8_gemm(q, s, native, scale_d, N, acc=acc, kernel=kernel)
     torch.cuda.synchronize()
     return (y.cpu().numpy(), acc.cpu().numpy() if with_acc else None, q.cpu().numpy(), s.cpu().numpy())
 
@@ -75,25 +75,30 @@ SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 5
          (1600, 300, 512)]
 
 
+@pytest.mark.parametrize("kernel", ["auto", "tc", "gemv"])
 @pytest.mark.parametrize("M,N,K", SMALL)
-def test_w4a8_small_full(M, N, K):
+def test_w4a8_small_full(M, N, K, kernel):
+    if kernel == "gemv" and M > sbm.W4A8_GEMV_MAX_M:
+        pytest.skip("the GEMV serves M <= 4")
     W = synth.weights(0, 3, N, K, sigma=0.02)
     x = synth.activations(0, 3, M, K)
     y_o, acc_o, q_o, s_o, w4_o, S_o = oracle.w4a8_reference(x, W)
     native, scale_d, w4, scale = upload_w4(W)
     assert np.array_equal(w4, w4_o) and np.array_equal(scale, S_o)
-    y, acc, q, s = run_w4(x, native, scale_d, N)
+    y, acc, q, s = run_w4(x, native, scale_d, N, kernel=kernel)
     assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
     assert np.array_equal(acc, acc_o)
     assert_y_close(y, y_o)
-    y2, _, _, _ = run_w4(x, native, scale_d, N, with_acc=False)     # y only: TMA stores of whole tiles
+    y2, _, _, _ = run_w4(x, native, scale_d, N, with_acc=False, kernel=kernel)   # y only (TMA stores on tc)
     assert np.array_equal(y2, y)
 
 
-def test_w4a8_extreme_values_near_int32():
+@pytest.mark.parametrize("M", [3, 20])
+def test_w4a8_extreme_values_near_int32(M):
     """w = -8 (bit pattern 1000, not produced by the quantiser) and q = +-127
-    at K = 14336: the x16 sums reach -127 * 128 * K = -2.3e8."""
-    N, K, M = 256, 14336, 20
+    at K = 14336: the x16 sums reach -127 * 128 * K = -2.3e8 (M = 3 runs the
+    GEMV, M = 20 the tensor-core kernel)."""
+    N, K = 256, 14336
     w4 = np.full((N, K // 2), 0x88, dtype=np.uint8)            # every weight -8
     w4[1::2] = 0x77                                             # odd rows: +7
     native = sbm.w4a8_repack(torch.from_numpy(w4).cuda(), N, K)
@@ -112,10 +117,11 @@ def test_w4a8_extreme_values_near_int32():
     assert_y_close(y.cpu().numpy(), oracle.w4a8_epilogue(acc_o, np.full(N, 0.5, np.float32), s_o))
 
 
-def test_w4a8_zero_token_and_repeat():
+@pytest.mark.parametrize("M", [3, 5])
+def test_w4a8_zero_token_and_repeat(M):
     N, K = 300, 1024
     W = synth.weights(0, 4, N, K)
-    x = synth.activations(0, 4, 5, K)
+    x = synth.activations(0, 4, M, K)
     x[2] = 0.0
     native, scale_d, _, _ = upload_w4(W)
     first = run_w4(x, native, scale_d, N)
@@ -125,8 +131,10 @@ def test_w4a8_zero_token_and_repeat():
         assert np.array_equal(again[1], first[1]) and np.array_equal(again[0], first[0])
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 4096, 14336), (8, 14336, 4096), (2048, 4096, 14336), (2048, 14336, 4096)])
-def test_w4a8_full_size_sampled(M, K, N):
+@pytest.mark.parametrize("M,K,N,kernel", [(1, 4096, 14336, "auto"), (1, 4096, 14336, "tc"), (4, 14336, 4096, "auto"),
+                                          (8, 14336, 4096, "auto"), (2048, 4096, 14336, "auto"),
+                                          (2048, 14336, 4096, "auto")])
+def test_w4a8_full_size_sampled(M, K, N, kernel):
     cfg = 1 if M == 1 else (2 if M <= 32 else 3)
     W = synth.config_weights(cfg, 0, K, N)
     native, scale_d, w4, scale = upload_w4(W)
@@ -136,11 +144,11 @@ def test_w4a8_full_size_sampled(M, K, N):
     x = synth.config_activations(cfg, 0, M, K)
     q_o, s_o = oracle.quant_act(x)
     acc_o = oracle.w4a8_gemm(q_o, w4[rows], K)
-    y, acc, q, s = run_w4(x, native, scale_d, N)
+    y, acc, q, s = run_w4(x, native, scale_d, N, kernel=kernel)
     assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
     assert np.array_equal(acc[:, rows], acc_o)
     assert_y_close(y[:, rows], oracle.w4a8_epilogue(acc_o, S_rows, s_o))
-    y2, _, _, _ = run_w4(x, native, scale_d, N, with_acc=False)
+    y2, _, _, _ = run_w4(x, native, scale_d, N, with_acc=False, kernel=kernel)
     assert np.array_equal(y2, y)
     if M > 16:
         Wq_full = oracle.w4a8_unpack(w4, K)

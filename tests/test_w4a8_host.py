@@ -69,3 +69,10 @@ def test_w4a8_argument_errors(lib):
     assert L.sherry_w4a8_gemm_acc(fake, fake, fake, fake, None, None, 1, 1, 32, None) == sbm.ERR_INVALID_ARG
     assert L.sherry_w4a8_gemm(ctypes.c_void_p((1 << 20) + 4), fake, fake, fake, fake, 1, 1, 32, None) == \
         sbm.ERR_INVALID_ARG
+    # the GEMV serves M <= 4 only; both explicit kernels check shapes before launching
+    assert L.sherry_w4a8_gemm_gemv(fake, fake, fake, fake, fake, None, sbm.W4A8_GEMV_MAX_M + 1, 1, 32, None) == \
+        sbm.ERR_UNSUPPORTED_SHAPE
+    assert L.sherry_w4a8_gemm_gemv(fake, fake, fake, fake, fake, None, 1, 1, 132128, None) == \
+        sbm.ERR_UNSUPPORTED_SHAPE
+    assert L.sherry_w4a8_gemm_tc(fake, fake, fake, fake, fake, None, 1, 1, 48, None) == sbm.ERR_UNSUPPORTED_SHAPE
+    assert L.sherry_w4a8_gemm_tc(None, fake, fake, fake, fake, None, 1, 1, 32, None) == sbm.ERR_INVALID_ARG

@@ -42,6 +42,8 @@ static int check(int64_t N, int64_t K)
                 for (int q = 0; q < 4; ++q) {
                     const uint8_t* piece = blk + q * SHERRY_TILE_ROWS * 16 + 16 * row;
                     if (piece != blk + 4 * sherry_w4_word_index(q, row, 0)) return 10;
+                    // the GEMV kernel's address of the same piece
+                    if (piece != bytes + sherry_w4_piece_offset(n, Kc, 4 * c + q)) return 12;
                     for (int i = 0; i < 4; ++i) {
                         uint32_t v = 0;
                         for (int b = 0; b < 4; ++b) v |= (uint32_t)piece[4 * i + b] << (8 * b);
