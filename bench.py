@@ -602,8 +602,8 @@ def w4a8_extras(args, flush, int8_peak, lib_tops, world):
     import torch
     import sparse_bit_matmul_b200 as sbm
     import synth
-    out = {"kernel": "sherry_w4a8_gemm: w4a8_gemv_kernel (CUDA cores) for M <= 4, "
-                     "sherry_gemm_tc_kernel<BN, SC, int4 weights> above",
+    out = {"kernel": "sherry_w4a8_gemm: sherry_gemm_tc_kernel<BN, SC, int4 weights> for every M; "
+                     "small M also timed on the CUDA-core comparison GEMV (sherry_w4a8_gemm_gemv)",
            "weights": "synthetic N(0, 0.02) quantised per channel to SINT4 (S = max|w| / 7)"}
     K, N = 4096, 14336
     copies = 9                                    # 9 x 29.4 MB = 264 MB > 2 x L2
@@ -612,18 +612,19 @@ def w4a8_extras(args, flush, int8_peak, lib_tops, world):
         w4, scale = sbm.w4a8_pack(synth.config_weights(1, c, K, N))
         mats.append((sbm.w4a8_repack(torch.from_numpy(w4).cuda(), N, K), torch.from_numpy(scale).cuda()))
     small = {}
-    for M in (1, 4, 16):
+    for M, kern in ((1, "auto"), (4, "auto"), (16, "auto"), (1, "gemv"), (4, "gemv")):
         q, s = sbm.quant_act(torch.from_numpy(synth.config_activations(2, 0, M, K)).cuda())
         y = torch.empty((M, N), device="cuda")
 
         def fn():
             for nat, sc in mats:
-                sbm.w4a8_gemm(q, s, nat, sc, N, out=y)
+                sbm.w4a8_gemm(q, s, nat, sc, N, out=y, kernel=kern)
         g = capture(fn)
         reps = max(3, args.steps // 4)
         t = max_over_ranks(time_graph(g, reps, 2, world), world)
         gbs = w4a8_bytes(M, K, N) * copies * reps / t / 1e9
-        small[str(M)] = {"gbs": round(gbs, 1), "us_per_call": round(t / (copies * reps) * 1e6, 2)}
+        key = str(M) if kern == "auto" else f"{M}_gemv"
+        small[key] = {"gbs": round(gbs, 1), "us_per_call": round(t / (copies * reps) * 1e6, 2)}
         del g
     out[f"small_M_K{K}_N{N}_rotation{copies}"] = small
     pre = {}

@@ -342,13 +342,13 @@ int sherry_w4a8_unpack(const uint8_t* w4, int64_t N, int64_t K, int8_t* Wq);
 int sherry_w4a8_repack(const uint8_t* w4_dev, int64_t N, int64_t K, void* native_dev,
                        void* stream);
 
-/* Largest M that sherry_w4a8_gemm sends to the CUDA-core GEMV. */
+/* Largest M the CUDA-core GEMV (sherry_w4a8_gemm_gemv) serves. */
 #define SHERRY_W4A8_GEMV_MAX_M 4
 
 /*
  * sherry_w4a8_gemm_acc -- device, asynchronous.  The W4A8 contraction and
- * dequantisation above.  M <= SHERRY_W4A8_GEMV_MAX_M runs
- * sherry_w4a8_gemm_gemv; larger M runs sherry_w4a8_gemm_tc.
+ * dequantisation above, for every M on the tensor-core kernel
+ * (sherry_w4a8_gemm_tc; it measured faster than the GEMV at M = 1 and 4).
  *   x_i8, x_scale  [in]  from sherry_quant_act, device memory (x_i8 16-byte aligned)
  *   W4native       [in]  from sherry_w4a8_repack, device memory, 16-byte aligned
  *   scale          [in]  fp32 [N] per-channel S from sherry_w4a8_pack, device memory
@@ -373,7 +373,8 @@ int sherry_w4a8_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* W4
 
 /*
  * sherry_w4a8_gemm_gemv -- device, asynchronous.  The same, for M <=
- * SHERRY_W4A8_GEMV_MAX_M, on the CUDA cores.  A CTA owns 32 rows and splits
+ * SHERRY_W4A8_GEMV_MAX_M, on the CUDA cores (a comparison kernel: the
+ * default path is the tensor-core kernel).  A CTA owns 32 rows and splits
  * K among its warps; the shift into int8 and dp4a run in registers.  Larger
  * M returns SHERRY_ERR_UNSUPPORTED_SHAPE.  Needs no workspace.  Arguments as
  * sherry_w4a8_gemm_acc.

@@ -297,7 +297,8 @@ def w4a8_gemm(x_i8, x_scale, w4_native, scale, N: int, out=None, acc=None, want_
               kernel: str = "auto"):
     """y fp32 [M][N] (and optionally the int32 sums after the division by 16)
     from int8 activations and kernel-native SINT4 weights.  kernel: "auto"
-    (the CUDA-core GEMV for M <= 4, tensor cores above), "tc" or "gemv"."""
+    (sherry_w4a8_gemm: the tensor-core kernel for every M), "tc" or "gemv"
+    (the CUDA-core comparison kernel, M <= 4)."""
     import torch
     M, K = x_i8.shape
     y = None

@@ -732,11 +732,12 @@ int sherry_w4a8_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* W4
     return launch_tc<192, 1, W4>(x_i8, x_scale, W4native, scale, y, acc, M, N, K, s);
 }
 
+// Every M runs on the tensor cores: at M = 1 and 4 (K=4096, N=14336) the
+// CUDA-core GEMV measured 11.5 and 20.0 us per call against about 9.3-10.2
+// us for the tensor-core kernel.
 int sherry_w4a8_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* W4native, const float* scale,
                          float* y, int32_t* acc, int64_t M, int64_t N, int64_t K, void* stream)
 {
-    if (M >= 1 && M <= SHERRY_W4A8_GEMV_MAX_M)
-        return sherry_w4a8_gemm_gemv(x_i8, x_scale, W4native, scale, y, acc, M, N, K, stream);
     return sherry_w4a8_gemm_tc(x_i8, x_scale, W4native, scale, y, acc, M, N, K, stream);
 }
 

@@ -9,9 +9,10 @@
 // the native layout, and the products are summed with dp4a.
 //
 // With one to four tokens the weights are read once and each weight byte
-// meets at most 8 multiply-adds: the launch is bound by HBM, not by the
-// tensor pipe, so it does not go through the tcgen05 pipeline and its role
-// hand-offs.  A CTA owns 32 consecutive rows (lane = row: a warp's 16-byte
+// meets at most 8 multiply-adds, so this kernel skips the tcgen05 pipeline
+// and its role hand-offs.  It is a comparison kernel: at K=4096, N=14336 it
+// measured 11.5 us (M=1) and 20.0 us (M=4) per call, slower than the
+// tensor-core kernel, which stays the default for every M.  A CTA owns 32 consecutive rows (lane = row: a warp's 16-byte
 // loads of one piece cover 512 contiguous bytes of the native layout) and
 // its PARTS warps split K into equal runs of 32-weight pieces; the partial
 // sums meet in shared memory and the first MT warps write the outputs.

@@ -93,11 +93,11 @@ def test_w4a8_small_full(M, N, K, kernel):
     assert np.array_equal(y2, y)
 
 
-@pytest.mark.parametrize("M", [3, 20])
-def test_w4a8_extreme_values_near_int32(M):
+@pytest.mark.parametrize("M,kernel", [(3, "gemv"), (3, "auto"), (20, "auto")])
+def test_w4a8_extreme_values_near_int32(M, kernel):
     """w = -8 (bit pattern 1000, not produced by the quantiser) and q = +-127
-    at K = 14336: the x16 sums reach -127 * 128 * K = -2.3e8 (M = 3 runs the
-    GEMV, M = 20 the tensor-core kernel)."""
+    at K = 14336: the x16 sums reach -127 * 128 * K = -2.3e8, on the CUDA-core
+    GEMV and on the tensor-core kernel."""
     N, K = 256, 14336
     w4 = np.full((N, K // 2), 0x88, dtype=np.uint8)            # every weight -8
     w4[1::2] = 0x77                                             # odd rows: +7
@@ -111,27 +111,28 @@ def test_w4a8_extreme_values_near_int32(M):
     xd = torch.from_numpy(x).cuda()
     q, s = sbm.quant_act(xd)
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
-    y = sbm.w4a8_gemm(q, s, native, scale_d, N, acc=acc)
+    y = sbm.w4a8_gemm(q, s, native, scale_d, N, acc=acc, kernel=kernel)
     torch.cuda.synchronize()
     assert np.array_equal(acc.cpu().numpy(), acc_o)
     assert_y_close(y.cpu().numpy(), oracle.w4a8_epilogue(acc_o, np.full(N, 0.5, np.float32), s_o))
 
 
-@pytest.mark.parametrize("M", [3, 5])
-def test_w4a8_zero_token_and_repeat(M):
+@pytest.mark.parametrize("M,kernel", [(3, "gemv"), (3, "auto"), (5, "auto")])
+def test_w4a8_zero_token_and_repeat(M, kernel):
     N, K = 300, 1024
     W = synth.weights(0, 4, N, K)
     x = synth.activations(0, 4, M, K)
     x[2] = 0.0
     native, scale_d, _, _ = upload_w4(W)
-    first = run_w4(x, native, scale_d, N)
+    first = run_w4(x, native, scale_d, N, kernel=kernel)
     assert np.all(first[0][2] == 0) and np.all(first[1][2] == 0)
     for _ in range(3):
-        again = run_w4(x, native, scale_d, N)
+        again = run_w4(x, native, scale_d, N, kernel=kernel)
         assert np.array_equal(again[1], first[1]) and np.array_equal(again[0], first[0])
 
 
-@pytest.mark.parametrize("M,K,N,kernel", [(1, 4096, 14336, "auto"), (1, 4096, 14336, "tc"), (4, 14336, 4096, "auto"),
+@pytest.mark.parametrize("M,K,N,kernel", [(1, 4096, 14336, "auto"), (1, 4096, 14336, "gemv"),
+                                          (4, 14336, 4096, "auto"), (4, 14336, 4096, "gemv"),
                                           (8, 14336, 4096, "auto"), (2048, 4096, 14336, "auto"),
                                           (2048, 14336, 4096, "auto")])
 def test_w4a8_full_size_sampled(M, K, N, kernel):
