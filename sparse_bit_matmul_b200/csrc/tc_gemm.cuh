@@ -259,38 +259,6 @@ __device__ __forceinline__ void report(unsigned* status, volatile int* abort_fla
     *abort_flag = 1;
 }
 
-// The sequence of stages of one CTA: its unit range [u0, u1) cut at tile ends
-// into segments, each segment into stages of at most SC chunks.  Every role
-// walks this same sequence.
-template <int SC>
-struct StageWalk {
-    int64_t u, u1, Kc, tile, tile_end;
-    __device__ StageWalk(int64_t u0_, int64_t u1_, int64_t Kc_) : u(u0_), u1(u1_), Kc(Kc_)
-    {
-        tile = u0_ / Kc_;
-        tile_end = (tile + 1) * Kc_;
-    }
-    __device__ bool done() const { return u >= u1; }
-    __device__ int64_t seg_end() const { return tile_end < u1 ? tile_end : u1; }
-    __device__ int64_t chunk() const { return u - tile * Kc; }
-    __device__ int nch() const
-    {
-        const int64_t left = seg_end() - u;
-        return left < SC ? (int)left : SC;
-    }
-    // advance past the current stage; returns true when a segment ended
-    __device__ bool next()
-    {
-        u += nch();
-        if (u >= tile_end || u >= u1) {
-            ++tile;
-            tile_end += Kc;
-            return true;
-        }
-        return false;
-    }
-};
-
 template <int BN, int SC, int WF = kWeightSherry>
 __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
     sherry_gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap,
