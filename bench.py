@@ -226,6 +226,38 @@ def cpu_baseline(seconds: float, copy: int = 0):
                       f"(activation quantiser + unpack + int contraction + epilogue), {el:.1f} s"}
 
 
+def cpu_lut_baseline(seconds: float, copy: int = 0):
+    """The page's own CPU scheme (cpu_lut: 16-entry segment tables read with
+    vpshufb, sign, integer sums, one float scaling) on the host cores, on
+    the same bounded sample as cpu_baseline; int8 activations and the
+    lookup layout are prepared before the timed passes."""
+    try:
+        import cpu_lut
+        import oracle
+        import sparse_bit_matmul_b200 as sbm
+        import synth
+        layers = []
+        for K, N in PROJ_SHAPES:
+            codes, alpha = sbm.pack(synth.config_weights(1, copy, K, N))
+            q, s = oracle.quant_act(synth.config_activations(1, copy, 1, K))
+            layers.append((K, N, cpu_lut.prepare(codes, K), alpha, q, s))
+        done_bytes, t0, passes = 0, time.perf_counter(), 0
+        while True:
+            for K, N, prep, alpha, q, s in layers:
+                cpu_lut.gemm(q, s, prep, alpha, N, K, want_acc=False)
+                done_bytes += algorithmic_bytes(1, K, N)
+            passes += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+        return {"value": round(done_bytes / el / 1e9, 3), "unit": "GB/s", "cores": cpu_lut.num_threads(),
+                "kind": "page_cpu_lut_" + ("avx2" if cpu_lut.has_avx2() else "scalar"),
+                "sample": f"{passes} pass(es) over the 3 projections of layer copy {copy} at M=1 "
+                          f"(table build + lookups + int sums + epilogue; int8 activations prepared), {el:.1f} s"}
+    except Exception as e:                      # a comparison line only: never fails the bench
+        return {"unavailable": f"{type(e).__name__}: {e}"}
+
+
 def run_reference(args, world, rank):
     """--impl reference: the CPU oracle on a bounded sample, same metric."""
     if rank != 0:
@@ -487,6 +519,7 @@ def run_gpu(args, world, rank, local):
         out["extra"] = extras(args, layers, kernel, peaks, peak_src, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        out["cpu_lut"] = cpu_lut_baseline(min(args.cpu_seconds, 3.0))
     return out
 
 

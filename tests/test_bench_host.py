@@ -70,3 +70,10 @@ def test_reference_arm_two_ranks_prints_one_line():
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_cpu_lut_leg_reports_a_rate():
+    r = bench.cpu_lut_baseline(0.2)
+    assert "unavailable" not in r, r
+    assert r["value"] > 0 and r["unit"] == "GB/s" and r["cores"] >= 1
+    assert r["kind"].startswith("page_cpu_lut_")
