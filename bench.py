@@ -619,7 +619,10 @@ def extras(args, layers, kernel, peaks, peak_src, world):
     res["int8_library_gemm_tops"] = {"value": round(lib_tops, 1), "how": "torch._int_mm 8192^3, 10 launches"}
     for v in pre.values():
         v["frac_of_library_int8"] = round(v["int_tops_dense_equiv"] / lib_tops, 4)
-    res["w4a8"] = w4a8_extras(args, flush, int8_peak, lib_tops, world)
+    try:                                        # a second workload: its failure is reported, not fatal
+        res["w4a8"] = w4a8_extras(args, flush, int8_peak, lib_tops, world)
+    except Exception as e:
+        res["w4a8"] = {"error": f"{type(e).__name__}: {e}"}
     return res
 
 
