@@ -320,3 +320,29 @@ def w4a8_gemm(x_i8, x_scale, w4_native, scale, N: int, out=None, acc=None, want_
         raise ValueError(kernel)
     _check(rc, f"sherry_w4a8_gemm[{kernel}]")
     return y
+
+
+class W4A8Linear:
+    """Weights of one W4A8 linear layer resident on the device.
+
+    ``W4A8Linear.from_weights(W)`` quantises and packs on the host
+    (sherry_w4a8_pack), copies the SINT4 rows and the channel scales to the
+    device and repacks them (sherry_w4a8_repack).  ``forward(x)`` quantises
+    the activations (sherry_quant_act) and runs the W4A8 GEMM
+    (sherry_w4a8_gemm), asynchronously on the current stream.
+    """
+
+    def __init__(self, w_native, scale, N: int, K: int):
+        self.w_native, self.scale, self.N, self.K = w_native, scale, N, K
+
+    @classmethod
+    def from_weights(cls, W: np.ndarray, device="cuda"):
+        import torch
+        w4, scale = w4a8_pack(W)
+        N, K = W.shape
+        w_native = w4a8_repack(torch.from_numpy(w4).to(device), N, K)
+        return cls(w_native, torch.from_numpy(scale).to(device), N, K)
+
+    def forward(self, x, out=None):
+        q, s = quant_act(x)
+        return w4a8_gemm(q, s, self.w_native, self.scale, self.N, out=out)

@@ -155,3 +155,15 @@ def test_w4a8_full_size_sampled(M, K, N, kernel):
         Wq_full = oracle.w4a8_unpack(w4, K)
         ref = torch._int_mm(torch.from_numpy(q_o).cuda(), torch.from_numpy(Wq_full).cuda().t().contiguous())
         assert torch.equal(torch.from_numpy(acc).cuda(), ref)
+
+
+def test_w4a8_linear_layer_object():
+    """W4A8Linear: host pack, device repack, quantiser + GEMM in forward()."""
+    N, K, M = 200, 1024, 3
+    W = synth.weights(0, 6, N, K)
+    x = synth.activations(0, 6, M, K)
+    y_o, *_ = oracle.w4a8_reference(x, W)
+    layer = sbm.W4A8Linear.from_weights(W, device="cuda")
+    y = layer.forward(torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    assert_y_close(y.cpu().numpy(), y_o)

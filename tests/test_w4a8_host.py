@@ -76,3 +76,21 @@ def test_w4a8_argument_errors(lib):
         sbm.ERR_UNSUPPORTED_SHAPE
     assert L.sherry_w4a8_gemm_tc(fake, fake, fake, fake, fake, None, 1, 1, 48, None) == sbm.ERR_UNSUPPORTED_SHAPE
     assert L.sherry_w4a8_gemm_tc(None, fake, fake, fake, fake, None, 1, 1, 32, None) == sbm.ERR_INVALID_ARG
+
+
+def test_w4a8_linear_wiring(lib, monkeypatch):
+    """W4A8Linear marshals the host pack, the device repack, the quantiser
+    and the GEMM in that order (device calls replaced by recorders)."""
+    import torch
+    calls = []
+    monkeypatch.setattr(sbm, "w4a8_repack", lambda w4_dev, N, K: calls.append(("repack", tuple(w4_dev.shape), N, K))
+                        or "native")
+    monkeypatch.setattr(sbm, "quant_act", lambda x: calls.append(("quant", tuple(x.shape))) or ("q", "s"))
+    monkeypatch.setattr(sbm, "w4a8_gemm", lambda q, s, nat, sc, N, out=None:
+                        calls.append(("gemm", q, s, nat, tuple(sc.shape), N, out)) or "y")
+    W = synth.weights(0, 7, 40, 96)
+    layer = sbm.W4A8Linear.from_weights(W, device="cpu")
+    w4, S = oracle.w4a8_pack(oracle.w4a8_quantise(W)[0]), oracle.w4a8_quantise(W)[1]
+    assert np.array_equal(layer.scale.numpy(), S) and (layer.N, layer.K) == (40, 96)
+    assert layer.forward(torch.zeros(3, 96)) == "y"
+    assert calls == [("repack", w4.shape, 40, 96), ("quant", (3, 96)), ("gemm", "q", "s", "native", (40,), 40, None)]
