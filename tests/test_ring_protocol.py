@@ -85,3 +85,63 @@ def test_whole_round_rings_never_read_a_stale_stage(S, G):
 @pytest.mark.parametrize("S,G", [(4, 3), (5, 3), (7, 3), (10, 3)])
 def test_other_rings_can_read_a_stale_stage(S, G):
     assert any(run_ring(S, G, 60, seed) > 0 for seed in range(400))
+
+
+def run_a_ring(A: int, G: int, iters: int, seed: int) -> int:
+    """The TMEM A-slot ring: decoder group g writes slot i mod A for its
+    iterations i = g (mod G) after a parity wait on aempty; the MMA reads the
+    slots in order and its commits complete in issue order, at random times.
+    Returns the number of overwrites of a slot an unfinished MMA still reads
+    (or of reads of a slot that does not hold the MMA's iteration)."""
+    rng = random.Random(seed)
+    aempty_done = [0] * A               # completed phases of aempty(a)
+    slot_tag = [-1] * A                 # iteration whose weights a slot holds
+    dec_next = list(range(G))
+    written = [False] * iters
+    mma_next = 0                        # next iteration the MMA issues
+    mma_done = 0                        # MMAs completed (in issue order)
+    bad = 0
+
+    def passes(done: int, k: int) -> bool:
+        return (done & 1) != (k & 1)
+
+    while mma_done < iters:
+        moves = []
+        for g in range(G):
+            i = dec_next[g]
+            # the wait for the slot's previous use (iteration i - A): phase i//A - 1
+            if i < iters and passes(aempty_done[i % A], i // A - 1):
+                moves.append(("dec", g))
+        if mma_next < iters and written[mma_next]:
+            moves.append("issue")
+        if mma_done < mma_next:
+            moves.append("complete")
+        if not moves:
+            return bad + 1000
+        mv = rng.choice(moves)
+        if mv == "issue":
+            if slot_tag[mma_next % A] != mma_next:
+                bad += 1
+            mma_next += 1
+        elif mv == "complete":
+            aempty_done[mma_done % A] += 1
+            mma_done += 1
+        else:
+            g = mv[1]
+            i = dec_next[g]
+            if i - A >= 0 and mma_done <= i - A:       # previous user of the slot still in flight
+                bad += 1
+            slot_tag[i % A] = i
+            written[i] = True
+            dec_next[g] += G
+    return bad
+
+
+@pytest.mark.parametrize("A,G", [(3, 3), (4, 3), (7, 3), (2, 2), (3, 2)])
+def test_a_ring_at_least_as_deep_as_the_groups_is_safe(A, G):
+    assert all(run_a_ring(A, G, 60, seed) == 0 for seed in range(400))
+
+
+@pytest.mark.parametrize("A,G", [(2, 3), (1, 2)])
+def test_a_ring_shallower_than_the_groups_is_not(A, G):
+    assert any(run_a_ring(A, G, 60, seed) > 0 for seed in range(400))
