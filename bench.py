@@ -55,10 +55,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["decode", "small", "prefill", "w4a8"], default=None,
+    ap.add_argument("--profile-case", choices=["decode", "small", "prefill", "w4a8", "long"], default=None,
                     help="run a few launches of one layer shape (K=4096, N=14336; M=1, 16 or 2048; "
-                         "w4a8: the SINT4 x int8 GEMM at M=2048) and exit: the target of the "
-                         "committed ncu captures")
+                         "w4a8: the SINT4 x int8 GEMM at M=2048; long: M=1, K=8192, N=28672) and exit: "
+                         "the target of the committed ncu captures")
     return ap.parse_args(argv)
 
 
@@ -197,17 +197,23 @@ def barrier(world: int):
 
 
 # ------------------------------------------------------------ CPU baseline
+def oracle_codes(W):
+    """The oracle's own ternarisation and packing (sec. 3.1, sec. 2.1): the
+    oracle-side legs never load the CUDA library."""
+    import oracle
+    T, alpha = oracle.quantise(W)
+    return oracle.pack(T), alpha
+
+
 def cpu_baseline(seconds: float, copy: int = 0):
     """The oracle as it stands on a bounded sample: unpack + contract +
     epilogue (and the activation quantiser) over the three projections of
     one layer copy, repeated until ~`seconds` of CPU work."""
     import oracle
-    import sparse_bit_matmul_b200 as sbm
     import synth
     layers = []
     for K, N in PROJ_SHAPES:
-        W = synth.config_weights(1, copy, K, N)
-        codes, alpha = sbm.pack(W)
+        codes, alpha = oracle_codes(synth.config_weights(1, copy, K, N))
         x = synth.config_activations(1, copy, 1, K)
         layers.append((K, N, codes, alpha, x))
     done_bytes, t0, passes = 0, time.perf_counter(), 0
@@ -234,11 +240,10 @@ def cpu_lut_baseline(seconds: float, copy: int = 0):
     try:
         import cpu_lut
         import oracle
-        import sparse_bit_matmul_b200 as sbm
         import synth
         layers = []
         for K, N in PROJ_SHAPES:
-            codes, alpha = sbm.pack(synth.config_weights(1, copy, K, N))
+            codes, alpha = oracle_codes(synth.config_weights(1, copy, K, N))
             q, s = oracle.quant_act(synth.config_activations(1, copy, 1, K))
             layers.append((K, N, cpu_lut.prepare(codes, K), alpha, q, s))
         done_bytes, t0, passes = 0, time.perf_counter(), 0
@@ -250,8 +255,13 @@ def cpu_lut_baseline(seconds: float, copy: int = 0):
             el = time.perf_counter() - t0
             if el >= seconds:
                 break
+        working_set = sum(prep.nbytes + alpha.nbytes + q.nbytes for _, _, prep, alpha, q, _ in layers)
         return {"value": round(done_bytes / el / 1e9, 3), "unit": "GB/s", "cores": cpu_lut.num_threads(),
                 "kind": "page_cpu_lut_" + ("avx2" if cpu_lut.has_avx2() else "scalar"),
+                "working_set_bytes": int(working_set),
+                "cache_resident": ("possibly: one layer copy (%.0f MB in the lookup layout) is rotated, which may "
+                                   "fit the host's last-level cache; the GPU line streams 671 MB from HBM"
+                                   % (working_set / 1e6)),
                 "sample": f"{passes} pass(es) over the 3 projections of layer copy {copy} at M=1 "
                           f"(table build + lookups + int sums + epilogue; int8 activations prepared), {el:.1f} s"}
     except Exception as e:                      # a comparison line only: never fails the bench
@@ -263,12 +273,10 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     import oracle
-    import sparse_bit_matmul_b200 as sbm
     import synth
     layers = []
     for K, N in PROJ_SHAPES:
-        W = synth.config_weights(1, 0, K, N)
-        codes, alpha = sbm.pack(W)
+        codes, alpha = oracle_codes(synth.config_weights(1, 0, K, N))
         layers.append((K, N, codes, alpha, synth.config_activations(1, 0, 1, K)))
 
     def step(i):
@@ -466,7 +474,7 @@ def run_gpu(args, world, rank, local):
     t_dom = t_step if fused else t_gemm
     dom_launch_s = t_dom / (args.steps * n_launch)
     achieved = step_bytes / (t_dom / args.steps) / 1e9
-    dom_name = "sherry_decode_kernel<1,fused>" if fused else f"sherry_gemm_{kernel}"
+    dom_name = "sherry_decode_kernel<1,true,RT>" if fused else f"sherry_gemm_{kernel}"
     traffic = load_traffic(dom_name, step_bytes / n_launch)
     h2d = sum(L["x"].numel() * 4 for L in layers)
     d2h = sum(L["y"].numel() * 4 for L in layers)
@@ -516,7 +524,8 @@ def run_gpu(args, world, rank, local):
     }
     del g_step, g_gemm, g_quant, g_two, g_e2e, g_e2e_layer
     if not args.no_extras:
-        out["extra"] = extras(args, layers, kernel, peaks, peak_src, world)
+        out["extra"] = extras(args, layers, kernel, peaks, peak_src, world,
+                              sm_mhz=(clocks or {}).get("sm_mhz"))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
         out["cpu_lut"] = cpu_lut_baseline(min(args.cpu_seconds, 3.0))
@@ -540,12 +549,163 @@ def load_traffic(kernel: str, avg_algorithmic_bytes: float):
         return None
 
 
-def extras(args, layers, kernel, peaks, peak_src, world):
+def timed_single_launches(fn, flush, reps: int = 5):
+    """Median of `reps` single launches of fn, each after an L2 flush (CUDA
+    events on the current stream)."""
+    import torch
+    for _ in range(3):
+        fn()
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    return statistics.median(times)
+
+
+def device_copies(native, alpha, count: int):
+    """`count` weight copies on the device: the given ones first, then device
+    clones of them (distinct memory, so every launch streams its own bytes)."""
+    out = list(zip(native, alpha))
+    i = 0
+    while len(out) < count:
+        nat, al = out[i % len(native)]
+        out.append((nat.clone(), al))
+        i += 1
+    return out
+
+
+def gemm_tops_line(M, K, N, cfg, flush, int8_peak, kernel):
+    """One GEMM of config `cfg`'s distributions through sherry_gemm (int8
+    activations already quantised): single launches after an L2 flush;
+    int-TOPS counted as 2 M N K dense-equivalent operations."""
+    import torch
+    import sparse_bit_matmul_b200 as sbm
+    import synth
+    codes, alpha = sbm.pack(synth.config_weights(cfg, 0, K, N))
+    native = sbm.repack(torch.from_numpy(codes).cuda(), N, K)
+    al = torch.from_numpy(alpha).cuda()
+    q, s = sbm.quant_act(torch.from_numpy(synth.config_activations(cfg, 0, M, K)).cuda())
+    y = torch.empty((M, N), device="cuda")
+    t = timed_single_launches(lambda: sbm.gemm(q, s, native, al, N, out=y, kernel=kernel), flush)
+    tops = 2.0 * M * N * K / t / 1e12
+    return {"us": round(t * 1e6, 2), "int_tops_dense_equiv": round(tops, 1),
+            "frac_of_int8_peak": round(tops / int8_peak, 4), "frac_of_4500_spec": round(tops / 4500.0, 4),
+            "algorithmic_add_tops": round(0.75 * M * N * K / t / 1e12, 1)}
+
+
+def config4_m1_l2_resident(args, world, hbm_peak):
+    """Config 4 at M = 1: one 36.7 MB weight matrix called back to back, so
+    its codes stay in L2 (126 MB); labelled as such, not an HBM figure."""
+    import torch
+    import sparse_bit_matmul_b200 as sbm
+    import synth
+    K, N = 8192, 28672
+    codes, alpha = sbm.pack(synth.config_weights(4, 0, K, N))
+    native = sbm.repack(torch.from_numpy(codes).cuda(), N, K)
+    al = torch.from_numpy(alpha).cuda()
+    x = torch.from_numpy(synth.config_activations(4, 0, 1, K)).cuda()
+    y = torch.empty((1, N), device="cuda")
+
+    def fn():
+        for _ in range(8):
+            sbm.linear(x, native, al, N, out=y)
+    g = capture(fn)
+    reps = max(3, args.steps // 20)
+    t = max_over_ranks(time_graph(g, reps, 2, world), world)
+    call = t / (8 * reps)
+    gbs = algorithmic_bytes(1, K, N) / call / 1e9
+    return {"us_per_call": round(call * 1e6, 3), "gbs": round(gbs, 1),
+            "l2_resident": "36.7 MB of codes called back to back: served from L2, not HBM",
+            "frac_of_hbm_peak_for_context": round(gbs / hbm_peak, 4)}
+
+
+def decode_per_shape(args, world, hbm_peak):
+    """M = 1 through sherry_linear, one projection shape at a time, repeated
+    over device copies of at least 600 MB per shape (every weight byte from
+    HBM): us per call, GB/s and fraction of the HBM peak."""
+    import torch
+    import sparse_bit_matmul_b200 as sbm
+    import synth
+    out = {}
+    for K, N in PROJ_SHAPES:
+        per = N * K * 5 // 32
+        count = max(16, -(-600_000_000 // per))
+        base_n, base_a = [], []
+        for c in range(4):
+            codes, alpha = sbm.pack(synth.config_weights(1, c, K, N))
+            base_n.append(sbm.repack(torch.from_numpy(codes).cuda(), N, K))
+            base_a.append(torch.from_numpy(alpha).cuda())
+        mats = device_copies(base_n, base_a, count)
+        x = torch.from_numpy(synth.config_activations(1, 0, 1, K)).cuda()
+        y = torch.empty((1, N), device="cuda")
+
+        def fn():
+            for nat, al in mats:
+                sbm.linear(x, nat, al, N, out=y)
+        g = capture(fn)
+        reps = max(3, args.steps // 20)
+        t = max_over_ranks(time_graph(g, reps, 2, world), world)
+        call = t / (reps * count)
+        gbs = algorithmic_bytes(1, K, N) / call / 1e9
+        out[f"K{K}_N{N}"] = {"us_per_call": round(call * 1e6, 3), "gbs": round(gbs, 1),
+                             "frac": round(gbs / hbm_peak, 4), "copies": count}
+        del g, mats, base_n
+        torch.cuda.empty_cache()
+    return out
+
+
+def long_call(args, world, hbm_peak, sm_mhz):
+    """One long M = 1 call (K = 8192 -> N = 28672, 36.7 MB of codes) through
+    sherry_linear, rotated over 16 device copies (587 MB > L2): the
+    throughput the decode kernel sustains once per-call latency is a small
+    part of the call.  groups_per_sm_clock = (N K / 4) / (time x SMs x SM
+    clock), with the clock measured in the headline's timed window."""
+    import torch
+    import sparse_bit_matmul_b200 as sbm
+    import synth
+    K, N, copies = 8192, 28672, 16
+    base_n, base_a = [], []
+    for c in range(2):
+        codes, alpha = sbm.pack(synth.config_weights(4, c, K, N))
+        base_n.append(sbm.repack(torch.from_numpy(codes).cuda(), N, K))
+        base_a.append(torch.from_numpy(alpha).cuda())
+    mats = device_copies(base_n, base_a, copies)
+    x = torch.from_numpy(synth.config_activations(4, 0, 1, K)).cuda()
+    y = torch.empty((1, N), device="cuda")
+
+    def fn():
+        for nat, al in mats:
+            sbm.linear(x, nat, al, N, out=y)
+    g = capture(fn)
+    reps = max(3, args.steps // 20)
+    t = max_over_ranks(time_graph(g, reps, 2, world), world)
+    call = t / (reps * copies)
+    gbs = algorithmic_bytes(1, K, N) / call / 1e9
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    res = {"shape": "M=1, K=8192 -> N=28672 (config 4's projection), sherry_linear",
+           "copies": copies, "bytes_per_pass": algorithmic_bytes(1, K, N) * copies,
+           "us_per_call": round(call * 1e6, 3), "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)}
+    if sm_mhz:
+        res["groups_per_sm_clock"] = round((N * K / 4) / (call * sms * sm_mhz * 1e6), 2)
+        res["sm_mhz_used"] = sm_mhz
+    del g, mats, base_n
+    torch.cuda.empty_cache()
+    return res
+
+
+def extras(args, layers, kernel, peaks, peak_src, world, sm_mhz=None):
     import torch
     import sparse_bit_matmul_b200 as sbm
     import synth
     res = {}
-    # small-batch decode on the same weights (M = 4, 8, 16, 32)
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    # small-batch decode on the same weights (M = 4, 8, 16, 32): the public
+    # call, sherry_linear from fp32 activations (or the named GEMM kernel)
     small = {}
     for M in (4, 8, 16, 32):
         xs, xf = {}, {}
@@ -558,49 +718,41 @@ def extras(args, layers, kernel, peaks, peak_src, world):
 
         def fn():
             for L in layers:
-                q, s = xs[L["K"]]
                 if kernel == "auto":
-                    sbm.quant_act(xf[L["K"]], q, s)
-                sbm.gemm(q, s, L["native"], L["alpha"], L["N"], out=ys[L["N"]], kernel=kernel)
+                    sbm.linear(xf[L["K"]], L["native"], L["alpha"], L["N"], out=ys[L["N"]])
+                else:
+                    q, s = xs[L["K"]]
+                    sbm.gemm(q, s, L["native"], L["alpha"], L["N"], out=ys[L["N"]], kernel=kernel)
         g = capture(fn)
-        t = max_over_ranks(time_graph(g, max(3, args.steps // 4), 2, world), world)
+        reps = max(3, args.steps // 4)
+        t = max_over_ranks(time_graph(g, reps, 2, world), world)
         nb = sum(algorithmic_bytes(M, L["K"], L["N"]) for L in layers)
-        small[str(M)] = round(nb * max(3, args.steps // 4) / t / 1e9, 2)
+        gbs = nb * reps / t / 1e9
+        small[str(M)] = {"gbs": round(gbs, 2), "frac": round(gbs / hbm_peak, 4),
+                         "us_per_call": round(t / (reps * len(layers)) * 1e6, 3)}
         del g
-    res["small_batch_decode_gbs"] = small
-    res["small_batch_step"] = ("sherry_quant_act + sherry_gemm (decode kernel for M <= 2, tensor cores above) "
-                               "per layer call"
+    res["small_batch_decode"] = small
+    res["small_batch_step"] = ("sherry_linear per layer call (fp32 activations in: the dispatch of the library)"
                                if kernel == "auto" else f"GEMM kernel {kernel} only")
+    res["decode_per_shape_M1"] = decode_per_shape(args, world, hbm_peak)
+    res["long_call_M1"] = long_call(args, world, hbm_peak, sm_mhz)
     # prefill GEMM, M = 2048 (L2 flushed between timed launches)
     int8_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * NOMINAL_INT8_OVER_BF16
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     pre = {}
     for K, N in [(4096, 14336), (14336, 4096)]:
-        M = 2048
-        W = synth.config_weights(3, 0, K, N)
-        codes, alpha = sbm.pack(W)
-        native = sbm.repack(torch.from_numpy(codes).cuda(), N, K)
-        al = torch.from_numpy(alpha).cuda()
-        q, s = sbm.quant_act(torch.from_numpy(synth.config_activations(3, 0, M, K)).cuda())
-        y = torch.empty((M, N), device="cuda")
-        for _ in range(3):
-            sbm.gemm(q, s, native, al, N, out=y, kernel=kernel)
-        times = []
-        for _ in range(5):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            sbm.gemm(q, s, native, al, N, out=y, kernel=kernel)
-            e1.record()
-            torch.cuda.synchronize()
-            times.append(e0.elapsed_time(e1) / 1e3)
-        t = statistics.median(times)
-        tops = 2.0 * M * N * K / t / 1e12
-        pre[f"K{K}_N{N}"] = {"us": round(t * 1e6, 1), "int_tops_dense_equiv": round(tops, 1),
-                             "frac_of_int8_peak": round(tops / int8_peak, 4),
-                             "frac_of_4500_spec": round(tops / 4500.0, 4),
-                             "algorithmic_add_tops": round(0.75 * M * N * K / t / 1e12, 1)}
+        pre[f"K{K}_N{N}"] = gemm_tops_line(2048, K, N, 3, flush, int8_peak, kernel)
     res["prefill_M2048"] = pre
+    # mid-size M on the tensor cores (64-, 128-token tiles), K = 4096 -> N = 14336
+    res["prefill_mid_M"] = {str(M): gemm_tops_line(M, 4096, 14336, 3, flush, int8_peak, kernel)
+                            for M in (64, 128, 512, 1024)}
+    # the heavy-tailed stress shape (K = 8192 -> N = 28672): M = 1 keeps its
+    # 36.7 MB of codes in the 126 MB L2 across back-to-back calls (labelled);
+    # M = 128 and 4096 are single launches after an L2 flush
+    c4 = {"M128": gemm_tops_line(128, 8192, 28672, 4, flush, int8_peak, kernel),
+          "M4096": gemm_tops_line(4096, 8192, 28672, 4, flush, int8_peak, kernel)}
+    c4["M1_l2_resident"] = config4_m1_l2_resident(args, world, hbm_peak)
+    res["config4_K8192_N28672"] = c4
     res["int8_peak_tops"] = {"value": round(int8_peak, 1),
                              "source": f"{peak_src} bf16_tflops x nominal int8/bf16 ratio 2"}
     # practical dense INT8 tensor throughput of the library GEMM on this machine
@@ -712,9 +864,9 @@ def profile_case(args):
         print(json.dumps({"profile_case": "w4a8", "M": M, "K": K, "N": N, "launches": 4,
                           "device_status": status}))
         return 0 if status == 0 else 1
-    M = {"decode": 1, "small": 16, "prefill": 2048}[args.profile_case]
-    K, N = 4096, 14336
-    copies = 8 if M <= 16 else 1
+    M = {"decode": 1, "small": 16, "prefill": 2048, "long": 1}[args.profile_case]
+    K, N = (8192, 28672) if args.profile_case == "long" else (4096, 14336)
+    copies = 2 if args.profile_case == "long" else (8 if M <= 16 else 1)
     layers = []
     for c in range(copies):
         codes, alpha = sbm.pack(synth.config_weights(1 if M <= 16 else 3, c, K, N))

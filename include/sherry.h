@@ -29,10 +29,18 @@
  * Ownership: the caller owns every buffer passed in.  Host functions take host
  * pointers; device functions take device pointers and a cudaStream_t passed
  * as void* (NULL = legacy default stream).  Device functions are asynchronous
- * on that stream; none of them synchronises.  The only device memory the
- * library allocates itself is one workspace per device for split-K partial
- * sums, created on the first sherry_gemm call that needs it, grown when a
- * larger problem arrives, and kept (all zero between calls) until exit.
+ * on that stream: none of them allocates, frees or synchronises.  The device
+ * memory the library owns is, per device:
+ *   - the workspace set aside by sherry_reserve (host, synchronous): the
+ *     split-K partial sums and arrival counters of the tensor-core kernel,
+ *     all zero between calls, and the int8 activations and scales that
+ *     sherry_linear uses when the caller passes none.  A call that needs more
+ *     than was reserved returns SHERRY_ERR_WORKSPACE and launches nothing;
+ *   - the fixed scratch array of sherry_gemm_noalloc and the device status
+ *     word, both in the library's own device image.
+ * Calls that use the reserved workspace share it: calls that may run at the
+ * same time on different streams of one device must not be issued
+ * (serialise them on one stream or with events).
  *
  * Errors: every function returns a sherry_status.  Argument errors are
  * reported before anything is launched.  SHERRY_ERR_CUDA means a CUDA call
@@ -57,7 +65,8 @@ typedef enum {
     SHERRY_ERR_UNSUPPORTED_SHAPE = 2, /* K % 32 != 0, or a size beyond the int32 index range */
     SHERRY_ERR_NONFINITE = 3,         /* NaN or Inf in W (sherry_pack) */
     SHERRY_ERR_CUDA = 4,              /* a CUDA runtime call failed */
-    SHERRY_ERR_DEVICE = 5             /* the device is not sm_100 or lacks a needed feature */
+    SHERRY_ERR_DEVICE = 5,            /* the device is not sm_100 or lacks a needed feature */
+    SHERRY_ERR_WORKSPACE = 6          /* the call needs more workspace than sherry_reserve set aside */
 } sherry_status;
 
 /* Short English text for a status value; never NULL. */
@@ -153,9 +162,8 @@ int sherry_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_i8, float* 
  *   Wnative  [in]  kernel-native codes from sherry_repack, device memory, 16-byte aligned
  *   alpha    [in]  fp32 [N], device memory
  *   y        [out] fp32 [M][N], device memory
- * Calls on the same device share the split-K workspace: calls that may run
- * at the same time on different streams must not be issued (serialise them
- * on one stream or with events).
+ * Uses the workspace set aside by sherry_reserve when its tensor-core launch
+ * splits a tile over several CTAs (SHERRY_ERR_WORKSPACE when too small).
  */
 int sherry_gemm(const int8_t* x_i8, const float* x_scale, const void* Wnative,
                 const float* alpha, float* y, int64_t M, int64_t N, int64_t K, void* stream);
@@ -208,8 +216,8 @@ int sherry_gemm_decode(const int8_t* x_i8, const float* x_scale, const void* Wna
  * results.  For M <= SHERRY_LINEAR_FUSED_MAX_M (one token) it is one launch
  * of the decode kernel that also quantises (every CTA reads the whole
  * activation row, takes its absmax and quantises it into its shared memory).
- * Other shapes run sherry_quant_act into a per-device buffer of the library
- * (allocated on first use, grown with a stream synchronisation) and then
+ * Other shapes run sherry_quant_act into x_i8 / x_scale (sherry_linear_ex),
+ * or into the activation buffer that sherry_reserve set aside, and then
  * sherry_gemm.
  *   x        [in]  fp32 [M][K], device memory, 16-byte aligned
  *   Wnative  [in]  kernel-native codes, device memory, 16-byte aligned
@@ -389,10 +397,48 @@ int sherry_w4a8_gemm(const int8_t* x_i8, const float* x_scale, const void* W4nat
                      void* stream);
 
 /*
+ * sherry_selftest_wait -- device, asynchronous.  A check of failure
+ * detection (no counterpart on the page): one warp waits, with the bounded
+ * wait every kernel of the library uses, for an mbarrier phase that nothing
+ * completes.  After limit_ns nanoseconds of wall time (1 to 10^9) the wait
+ * gives up, the kernel records 0x107 in the device status word (read with
+ * sherry_last_device_status) and returns; the context stays usable.  No
+ * copy is in flight and no tensor memory is held when it gives up.
+ */
+int sherry_selftest_wait(uint64_t limit_ns, void* stream);
+
+/*
+ * sherry_workspace_bytes -- host.  Device bytes that sherry_reserve(max_M,
+ * max_K) sets aside on the current device: the tensor-core kernel's split-K
+ * slots (one per SM, the token tile of max_M tokens x 128 rows of int32)
+ * and counters, plus max_M x max_K int8 activations and max_M scales for
+ * sherry_linear.  0 for non-positive sizes or an unsupported device.
+ */
+size_t sherry_workspace_bytes(int64_t max_M, int64_t max_K);
+
+/*
+ * sherry_reserve -- host, synchronous.  Sets aside, on the current device,
+ * the workspace of every later call with M <= max_M and K <= max_K (any N):
+ * sherry_gemm, sherry_gemm_acc, sherry_gemm_tc, sherry_linear(_ex) and the
+ * W4A8 tensor-core entry points.  Grows what an earlier call reserved (never
+ * shrinks it); when it grows it first waits for the device to be idle, then
+ * frees the old buffer, allocates and zero-fills the new one.  Call it before
+ * capturing a stream into a CUDA graph and before timing.  The asynchronous
+ * entry points never allocate: without enough workspace they return
+ * SHERRY_ERR_WORKSPACE.  Calls whose tensor-core launch splits no tile over
+ * several CTAs, the decode kernel (M <= SHERRY_DECODE_MAX_M), the fused
+ * sherry_linear launch and sherry_gemm_noalloc need no workspace.
+ */
+int sherry_reserve(int64_t max_M, int64_t max_K);
+
+/*
  * sherry_last_device_status -- host, synchronous (copies one word from the
  * current device).  0 when no kernel of this library has reported a bounded
  * wait running out since the last reset; otherwise a nonzero code naming the
- * wait.  reset != 0 clears it.
+ * wait.  reset != 0 clears it; when the word was nonzero the reset also waits
+ * for the device to be idle and zero-fills the reserved workspace again,
+ * since a launch that gave up may have left partial sums and arrival
+ * counters in it.  After a nonzero status, reset it before the next call.
  */
 int sherry_last_device_status(int reset);
 

@@ -19,24 +19,36 @@
  *                   ||T||_0 = 3; solution: keep the 3 largest |w| with their
  *                   signs
  *
- * Readings taken where the page is silent or garbled (each one is listed with
- * its reason in the design notes):
- *   - groups run along K, the reduction axis;
+ * Readings taken where the page is silent or garbled, each with its reason:
+ *   - groups run along K, the reduction axis: the page's 4-element activation
+ *     segments only line up with weight groups along K;
  *   - alpha is one scale per output row n: sum of kept |w| (fp64, ascending k)
- *     divided by 0.75*K, rounded once to fp32;
- *   - ties in |w|: the lowest index is the one zeroed;
- *   - sign of a kept weight: negative iff w < 0.0f (so -0.0 and +0.0 are +);
+ *     divided by 0.75*K, rounded once to fp32.  One fp32 alpha per group of
+ *     4 would cost 8 bit/weight against the page's 1.25, and with exactly 3
+ *     nonzeros per group ||T||^2 = 0.75 K is fixed, so this alpha and the
+ *     per-group choice of T minimise ||W - alpha T||^2 together;
+ *   - ties in |w|: the lowest index is the one zeroed (every choice gives the
+ *     same error; one is needed for bit-exact codes);
+ *   - sign of a kept weight: negative iff w < 0.0f (so -0.0 and +0.0 are +),
+ *     the plain IEEE comparison;
  *   - code = z | s0<<2 | s1<<3 | s2<<4, z = zeroed position, s_j = sign bit
- *     of the j-th kept position in ascending order (1 = negative);
+ *     of the j-th kept position in ascending order (1 = negative): the page
+ *     fixes only the size, 5 bits;
  *   - the page's (4-bit pattern, 1 dominant-sign bit) form is the bijection
- *     pattern4 = z | (s1^s0)<<2 | (s2^s0)<<3, sign = s0;
+ *     pattern4 = z | (s1^s0)<<2 | (s2^s0)<<3, sign = s0: a literal "which 3
+ *     of 4 are nonzero" mask gives only 8 states with the sign bit and cannot
+ *     hold the page's own mixed-sign example block [-1, 0, +1, -1];
  *   - row n's code stream starts at byte n*(5K/32); code j occupies stream
- *     bits [5j, 5j+5), least significant bit first; K % 32 == 0;
+ *     bits [5j, 5j+5), least significant bit first; K % 32 == 0 (rows of
+ *     whole bytes; every workload's K qualifies);
  *   - activations: per token absmax a; s = a/127 (fp32 division); q =
  *     clamp(rint(x/s), -127, 127) with round-half-to-even; a == 0 gives
- *     s = 0 and q = 0;
+ *     s = 0 and q = 0: the page gives no rule, and this is the plainest
+ *     symmetric one (it never produces -128);
  *   - y[m][n] = (float)((float)acc[m][n] * alpha[n]) * s[m], two separately
- *     rounded fp32 products in this order.
+ *     rounded fp32 products in this order: the page says one float scale at
+ *     the end; a fixed order keeps y reproducible bit for bit, and
+ *     float(acc) is exact because |acc| <= 127 * 0.75 K < 2^24.
  *
  * Compile with -ffp-contract=off so that no multiply-add is fused.
  */

@@ -24,21 +24,23 @@
  *                        conversion -7 = 1001 -> 1001 0000 = -112, and the
  *                        identity sum(A*W*16)/16 = sum(A*W)
  *
- * Readings taken where the page is silent (each one is listed with its reason
- * in the design notes):
+ * Readings taken where the page is silent, each with its reason:
  *   - gamma = beta = 1: the learnable clipping factors need calibration data,
  *     which this path does not have; "per-channel" = one S per output row n
  *     of W [N][K];
  *   - S = a / 7.0f in fp32 (a = max(|max_k W|, |min_k W|)), W_q =
  *     clamp(rint(W / S), -8, 7) with fp32 IEEE division and round half to
- *     even; a == 0 gives S = 0 and W_q = 0;
+ *     even; a == 0 gives S = 0 and W_q = 0: the page gives no rounding
+ *     rule, and these are the activation quantiser's rules;
  *   - activations: per-token absmax int8 (s = a / 127), the same quantiser as
  *     the Sherry path (oracle_quant_act);
  *   - storage: row n starts at byte n * K/2; byte j holds weight 2j in its
- *     low nibble and weight 2j+1 in its high nibble (two's complement);
+ *     low nibble and weight 2j+1 in its high nibble (two's complement): the
+ *     page shows single values only, and low-first matches the Sherry stream;
  *   - y[m][n] = (float)((float)acc[m][n] * S[n]) * s[m], two separately
  *     rounded fp32 products in this order, acc = the int32 sum after the
- *     division by 16.
+ *     division by 16: the same order as the Sherry epilogue, so y is
+ *     reproducible bit for bit.
  *
  * Compile with -ffp-contract=off so that no multiply-add is fused.
  */

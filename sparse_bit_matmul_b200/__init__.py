@@ -17,7 +17,7 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 SO_PATH = os.path.join(HERE, "libsherry_b200.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_NONFINITE, ERR_CUDA, ERR_DEVICE = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_NONFINITE, ERR_CUDA, ERR_DEVICE, ERR_WORKSPACE = range(7)
 
 # every entry point declared in include/sherry.h
 ABI_SYMBOLS = (
@@ -25,6 +25,7 @@ ABI_SYMBOLS = (
     "sherry_pack", "sherry_unpack", "sherry_repack", "sherry_quant_act", "sherry_gemm",
     "sherry_gemm_acc", "sherry_gemm_tc", "sherry_gemm_gemv", "sherry_gemm_simt", "sherry_gemm_noalloc",
     "sherry_gemm_decode", "sherry_linear", "sherry_linear_ex", "sherry_last_device_status",
+    "sherry_workspace_bytes", "sherry_reserve", "sherry_selftest_wait",
     "sherry_w4a8_packed_bytes", "sherry_w4a8_native_bytes", "sherry_w4a8_pack", "sherry_w4a8_unpack",
     "sherry_w4a8_repack", "sherry_w4a8_gemm", "sherry_w4a8_gemm_acc", "sherry_w4a8_gemm_tc",
     "sherry_w4a8_gemm_gemv",
@@ -69,6 +70,10 @@ def load() -> ctypes.CDLL:
     L.sherry_linear.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_linear_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.sherry_last_device_status.argtypes = [c_int]
+    L.sherry_workspace_bytes.argtypes = [i64, i64]
+    L.sherry_workspace_bytes.restype = ctypes.c_size_t
+    L.sherry_reserve.argtypes = [i64, i64]
+    L.sherry_selftest_wait.argtypes = [ctypes.c_uint64, vp]
     L.sherry_w4a8_packed_bytes.argtypes = [i64, i64]
     L.sherry_w4a8_packed_bytes.restype = ctypes.c_size_t
     L.sherry_w4a8_native_bytes.argtypes = [i64, i64]
@@ -140,6 +145,37 @@ def unpack(codes: np.ndarray, K: int) -> np.ndarray:
 
 
 # --------------------------------------------------------------- device side
+_reserved = {}          # device index -> (max_M, max_K) reserved through this binding
+
+
+def workspace_bytes(max_M: int, max_K: int) -> int:
+    """Device bytes sherry_reserve(max_M, max_K) sets aside on the current device."""
+    return int(load().sherry_workspace_bytes(max_M, max_K))
+
+
+def reserve(max_M: int, max_K: int, device=None):
+    """sherry_reserve on `device` (default: the current CUDA device): host-
+    synchronous; sets aside the workspace of every later call with
+    M <= max_M and K <= max_K.  Call it before capturing CUDA graphs."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    m0, k0 = _reserved.get(idx, (0, 0))
+    m1, k1 = max(m0, int(max_M)), max(k0, int(max_K))
+    if (m1, k1) != (m0, k0):
+        with torch.cuda.device(idx):
+            _check(load().sherry_reserve(m1, k1), "sherry_reserve")
+        _reserved[idx] = (m1, k1)
+
+
+def _ensure_workspace(t, M: int, K: int):
+    # the asynchronous entry points never allocate: the binding reserves (host,
+    # synchronous) the first time a call needs more than was set aside
+    m0, k0 = _reserved.get(t.device.index, (0, 0))
+    if M > m0 or K > k0:
+        reserve(M, K, t.device)
+
+
 def repack(codes_dev, N: int, K: int, out=None):
     """Canonical codes on the device -> kernel-native layout (uint8 tensor)."""
     import torch
@@ -177,6 +213,8 @@ def gemm(x_i8, x_scale, w_native, alpha, N: int, out=None, acc=None, want_y: boo
     if want_y:
         y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x_i8.device)
     L = load()
+    if kernel != "noalloc":
+        _ensure_workspace(x_i8, M, K)
     args = (_dptr(x_i8), _dptr(x_scale), _dptr(w_native), _dptr(alpha), _dptr(y), _dptr(acc), M, N, K,
             _stream(x_i8))
     if kernel == "auto":
@@ -211,6 +249,7 @@ def linear(x, w_native, alpha, N: int, out=None, acc=None, out_q=None, out_s=Non
     if want_y:
         y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
     L = load()
+    _ensure_workspace(x, M, K)
     if acc is None and out_q is None and out_s is None:
         rc = L.sherry_linear(_dptr(x), _dptr(w_native), _dptr(alpha), _dptr(y), M, N, K, _stream(x))
     else:
@@ -222,6 +261,16 @@ def linear(x, w_native, alpha, N: int, out=None, acc=None, out_q=None, out_s=Non
 
 def last_device_status(reset: bool = False) -> int:
     return int(load().sherry_last_device_status(1 if reset else 0))
+
+
+DEV_TIMEOUT_SELFTEST = 0x107   # device status code of sherry_selftest_wait
+
+
+def selftest_wait(limit_ns: int, stream=None):
+    """sherry_selftest_wait on the current stream: a bounded wait that runs out."""
+    import torch
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    _check(load().sherry_selftest_wait(int(limit_ns), st), "sherry_selftest_wait")
 
 
 class PackedLinear:
@@ -305,6 +354,7 @@ def w4a8_gemm(x_i8, x_scale, w4_native, scale, N: int, out=None, acc=None, want_
     if want_y:
         y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x_i8.device)
     L = load()
+    _ensure_workspace(x_i8, M, K)
     args = (_dptr(x_i8), _dptr(x_scale), _dptr(w4_native), _dptr(scale), _dptr(y), _dptr(acc), M, N, K,
             _stream(x_i8))
     if kernel == "auto":

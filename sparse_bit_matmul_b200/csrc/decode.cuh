@@ -11,22 +11,36 @@
 // every 5-bit code, one store of y.  The design keeps that chain short.
 //   * One CTA per SM (more only when its codes would not fit in shared
 //     memory), each owning a contiguous, balanced range of whole output rows
-//     over the full K: no split-K, no cross-CTA reduction, no atomics, no
-//     workspace, no clusters.
+//     over the full K: no split-K, no cross-CTA reduction, no atomics in
+//     global memory, no workspace, no clusters.
 //   * Before griddepcontrol.wait the CTA streams its rows' codes (the rotated
-//     word planes of the native layout) into shared memory with 4-byte
-//     cp.async copies: weights never depend on the previous kernel, so their
-//     fetch overlaps its decode.  The CTA lets the next kernel start only once
-//     its own activations are in shared memory, so that the next kernel's
-//     weight stream does not queue in front of those latency-critical reads.  The CTA is small enough in shared memory,
-//     threads and registers for the next layer's CTA to be resident at the
-//     same time and do the same.
+//     word planes of the native layout) into shared memory with 16-byte
+//     cp.async copies, and asks L2 to prefetch its share of the fp32
+//     activations (a prefetch has no effect on values, so it may run before
+//     the previous kernel has finished writing them).  Weights never depend
+//     on the previous kernel, so their fetch overlaps its decode.  The CTA
+//     lets the next kernel start only once its own activations are in
+//     shared memory, so that the next kernel's weight stream does not queue
+//     in front of those latency-critical reads.  The CTA is small enough in
+//     shared memory, threads and registers for the next layer's CTA to be
+//     resident at the same time and do the same.
 //   * After the wait every CTA reads the activations of its tokens (all of
-//     K), takes the absmax, quantises into shared memory; then thread
-//     (row i, K-part p) walks the chunks of its part: one 32-entry table
-//     load turns a code into int8x4 {-1,0,+1}, one dp4a per token adds it.
-//   * The K-parts of a row are summed in shared memory and the epilogue
-//     writes y (and acc) with coalesced stores.
+//     K), takes the absmax, quantises into shared memory.
+//   * Thread (row group i, K-part p) owns RT consecutive rows and walks the
+//     chunks of its part.  Per group: one 32-entry table load turns the
+//     5-bit code into int8x4 {-1,0,+1}, one dp4a per token adds it.  The
+//     shared-memory pipe is the limit of that loop (measured on B200: one
+//     conflict-free 32-bit lookup per clock per SM, a broadcast 128-bit
+//     activation load about 2.6 clocks): one 16-byte activation load serves
+//     all RT rows of a thread, so the table lookups are most of the pipe's
+//     work.  Consecutive lanes own consecutive row groups, so their code
+//     loads are consecutive 4*RT-byte pieces and their activation loads are
+//     broadcasts.  Activation chunks sit S >= 128 bytes apart, S chosen on
+//     the host so that the few K-parts that share a warp read different
+//     banks.
+//   * The K-parts of a row are summed in shared memory (every thread adds a
+//     share of the parts into the row's total with a shared atomic), and the
+//     epilogue writes y (and acc) with coalesced stores.
 #pragma once
 
 #include <cstdint>
@@ -41,6 +55,7 @@ namespace decode {
 constexpr int kMaxM = 8;
 constexpr int kMaxThreads = 512;
 constexpr int kSmemBudget = 100 * 1024;     // two CTAs (this layer, the next) per SM
+constexpr int kSmemBudgetMax = 200 * 1024;  // one CTA per SM: shapes whose activations alone need more
 constexpr int kXV = 8;                      // fused: float4 activations per thread held in registers
 
 struct Params {
@@ -56,26 +71,30 @@ struct Params {
     int64_t M, N, K, Kc;
     int G;                       // CTAs; CTA c owns rows [row_begin(c), row_begin(c+1))
     int R;                       // largest row count of a CTA, a multiple of 4
+    int Q;                       // row groups of RT rows: R / RT
     int P;                       // K-parts per row
     int CPT;                     // chunks per K-part
+    int S;                       // bytes between consecutive K chunks of the int8 activation buffer
 };
 
 // Shared memory: table | scales | warp maxima (two token slots) | partial sums [P][M][R] |
-// alpha [R] | codes [Kc][5][R] words | activations [M][Kc*128] int8.
+// row totals [M][R] | alpha [R] | codes [Kc][5][R] words | activations [M][Kc][S] int8.
 constexpr int kOffTable = 0;                              // 32 x u32, 128-byte aligned inside 256 bytes
 constexpr int kOffScale = 256;                            // [kMaxM] f32 s
 constexpr int kOffWarpMax = kOffScale + kMaxM * 4;        // [2][16 warps] f32
 constexpr int kOffRed = kOffWarpMax + 2 * 16 * 4;
 static_assert(kMaxThreads / 32 <= 16, "warp-maximum slots");
-__host__ __device__ inline int off_alpha(int M, int P, int R) { return (kOffRed + P * M * R * 4 + 15) & ~15; }
+static_assert(kOffRed % 16 == 0, "alignment");
+__host__ __device__ inline int off_sums(int M, int P, int R) { return (kOffRed + P * M * R * 4 + 15) & ~15; }
+__host__ __device__ inline int off_alpha(int M, int P, int R) { return (off_sums(M, P, R) + M * R * 4 + 15) & ~15; }
 __host__ __device__ inline int off_codes(int M, int P, int R) { return (off_alpha(M, P, R) + R * 4 + 15) & ~15; }
 __host__ __device__ inline int off_q(int M, int P, int R, int64_t Kc)
 {
     return (off_codes(M, P, R) + (int)Kc * SHERRY_CHUNK_WORDS * R * 4 + 15) & ~15;
 }
-__host__ __device__ inline int smem_bytes(int M, int P, int R, int64_t Kc)
+__host__ __device__ inline int smem_bytes(int M, int P, int R, int64_t Kc, int S)
 {
-    return off_q(M, P, R, Kc) + M * (int)Kc * SHERRY_KCHUNK;
+    return off_q(M, P, R, Kc) + M * (int)Kc * S;
 }
 
 __device__ __forceinline__ uint32_t expand_code(uint32_t c)
@@ -107,7 +126,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
+// L2 prefetch of a byte range (16-byte aligned start, size a multiple of 16)
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 // N consecutive 32-bit words from a shared address (aligned to 4 N bytes).
 template <int N>
@@ -128,22 +151,186 @@ __device__ __forceinline__ void lds_vec<4>(uint32_t addr, uint32_t (&v)[4])
     asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]) : "r"(addr));
 }
 
-template <int MT, bool FUSED>
+// Byte offset, in the table, of group g's code within a row's five chunk
+// words w[0..4] (w[5] = 0): (bits [5g, 5g+5)) * 4.  g is a compile-time
+// constant after unrolling, so this is one shift or funnel shift.
+template <int G>
+__device__ __forceinline__ uint32_t code_x4(const uint32_t (&w)[SHERRY_CHUNK_WORDS + 1])
+{
+    constexpr int bit = 5 * G, wi = bit >> 5, off = bit & 31;
+    uint32_t v;
+    if constexpr (off == 0) v = w[wi] << 2;
+    else if constexpr (off == 1) v = w[wi] << 1;
+    else if constexpr (off <= 27) v = w[wi] >> (off - 2);
+    else v = __funnelshift_r(w[wi], w[wi + 1], off - 2);
+    return v & 0x7Cu;
+}
+
+// The 4 groups of piece G4 (groups 4 G4 .. 4 G4 + 3) of RT rows: table entries.
+template <int G4, int RT>
+__device__ __forceinline__ void lookup_piece(const uint32_t (&w)[RT][SHERRY_CHUNK_WORDS + 1], uint32_t table_s,
+                                             uint32_t (&e)[RT][4])
+{
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        e[r][0] = ptx::lds_u32_nv(code_x4<4 * G4 + 0>(w[r]) | table_s);
+        e[r][1] = ptx::lds_u32_nv(code_x4<4 * G4 + 1>(w[r]) | table_s);
+        e[r][2] = ptx::lds_u32_nv(code_x4<4 * G4 + 2>(w[r]) | table_s);
+        e[r][3] = ptx::lds_u32_nv(code_x4<4 * G4 + 3>(w[r]) | table_s);
+    }
+}
+
+template <int G4, int MT, int RT>
+__device__ __forceinline__ void piece(const uint32_t (&w)[RT][SHERRY_CHUNK_WORDS + 1], uint32_t table_s,
+                                      uint32_t qc, int QK, int M, int32_t (&acc)[RT][MT])
+{
+    uint32_t e[RT][4];
+    lookup_piece<G4, RT>(w, table_s, e);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        if (m >= M) break;
+        uint32_t qv[4];
+        lds_vec<4>(qc + (uint32_t)(m * QK + 16 * G4), qv);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            int32_t a = acc[r][m];
+            a = __dp4a((int)e[r][0], (int)qv[0], a);
+            a = __dp4a((int)e[r][1], (int)qv[1], a);
+            a = __dp4a((int)e[r][2], (int)qv[2], a);
+            a = __dp4a((int)e[r][3], (int)qv[3], a);
+            acc[r][m] = a;
+        }
+    }
+}
+
+inline int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+inline int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+inline int min_i(int a, int b) { return a < b ? a : b; }
+
+// Work split of the decode kernel: G CTAs of at most R rows (one per SM
+// unless the codes of R rows would not fit the shared-memory budget), row
+// groups of RT rows (Q = R / RT of them), P K-parts of CPT chunks per row,
+// Q * P <= kMaxThreads.  RT is the largest that the token count's registers
+// allow and that still gives the CTA at least kMinBusyThreads working
+// threads.  False if even one row does not fit.
+struct Plan {
+    int G, R, RT, Q, P, CPT, threads, smem, S;
+};
+
+constexpr int kMinBusyThreads = 320;
+
+// Rows per thread that the registers allow for MT tokens: RT x MT
+// accumulators plus RT x 5 code words and RT x 4 table entries live at once.
+inline int rt_max(int64_t M) { return M <= 2 ? 4 : 2; }
+
+// Bytes between K chunks of the int8 activation buffer: 128 + 16 sigma.  The
+// K-parts that share a warp read their chunks at the same loop step; their
+// 16-byte pieces sit sigma * 4 * dc banks apart (dc: chunk distance), so
+// sigma is chosen to keep the pieces of a warp in different banks.
+inline int act_stride(int Q, int P, int CPT, int threads)
+{
+    int best = 0, best_bad = 1 << 30;
+    for (int sigma = 0; sigma < 8; ++sigma) {
+        const int S = 128 + 16 * sigma;
+        int bad = 0;
+        for (int w0 = 0; w0 < threads; w0 += 32) {
+            const int pa = w0 / Q, pb = min_i(P - 1, (w0 + 31) / Q);
+            for (int p1 = pa; p1 <= pb; ++p1)
+                for (int p2 = p1 + 1; p2 <= pb; ++p2) {
+                    const int banks = (int)(((int64_t)(p2 - p1) * CPT * S / 4) % 32);
+                    if (banks < 4 || banks > 28) ++bad;
+                }
+        }
+        if (bad < best_bad) {
+            best_bad = bad;
+            best = S;
+        }
+        if (bad == 0) break;
+    }
+    return best;
+}
+
+inline bool plan_within(int64_t N, int64_t Kc, int64_t M, int sms, int budget, Plan* out)
+{
+    // at least 4 rows per CTA: row boundaries rounded to 4 rows then leave no CTA empty
+    const int64_t gmax = max64(1, N / 4);
+    int64_t G = min64(sms, gmax);
+    const int rtmax = rt_max(M);
+    for (int iter = 0; iter < 64; ++iter) {
+        const int64_t R = ((N + G - 1) / G + 3 + 3) & ~int64_t(3);     // rounded groups, a multiple of 4
+        if (R > (int64_t)rtmax * kMaxThreads) {
+            // rows per CTA at most ceil(N / G) + 6 after rounding
+            const int64_t cap = (int64_t)rtmax * kMaxThreads - 8;
+            G = min64(gmax, max64(G + 1, (N + cap - 1) / cap));
+            continue;
+        }
+        int64_t RT = rtmax, Q = 0, P = 0, CPT = 0;
+        for (;; RT /= 2) {
+            Q = R / RT;
+            if (Q > kMaxThreads) return false;
+            P = max64(1, min64(Kc, kMaxThreads / Q));
+            CPT = (Kc + P - 1) / P;
+            P = (Kc + CPT - 1) / CPT;
+            if (Q * P >= kMinBusyThreads || RT == 1 || R / (RT / 2) > kMaxThreads) break;
+        }
+        const int threads = kMaxThreads;
+        for (int shrink = 0; shrink < 4; ++shrink) {
+            // the bank-spreading stride when it fits, else plain 128-byte chunks
+            int S = act_stride((int)Q, (int)P, (int)CPT, (int)(Q * P));
+            int64_t smem = smem_bytes((int)M, (int)P, (int)R, Kc, S);
+            if (smem > budget && S != SHERRY_KCHUNK) {
+                S = SHERRY_KCHUNK;
+                smem = smem_bytes((int)M, (int)P, (int)R, Kc, S);
+            }
+            if (smem <= budget) {
+                if (G > 0x7fffffff) return false;
+                out->G = (int)G;
+                out->R = (int)R;
+                out->RT = (int)RT;
+                out->Q = (int)Q;
+                out->P = (int)P;
+                out->CPT = (int)CPT;
+                out->threads = threads;
+                out->smem = (int)smem;
+                out->S = S;
+                return true;
+            }
+            if (P == 1) break;
+            CPT *= 2;                                                 // fewer K-parts: fewer partial sums
+            P = (Kc + CPT - 1) / CPT;
+        }
+        if (R <= 4 || G >= gmax) return false;
+        G = min64(gmax, 2 * G);                                       // about half the rows per CTA
+    }
+    return false;
+}
+
+// The plan of a launch: within kSmemBudget (two CTAs per SM, so the next
+// layer's CTA can start its weight fetch beside this one) when possible, else
+// within kSmemBudgetMax (one CTA per SM).
+inline bool plan(int64_t N, int64_t Kc, int64_t M, int sms, Plan* out)
+{
+    return plan_within(N, Kc, M, sms, kSmemBudget, out) || plan_within(N, Kc, M, sms, kSmemBudgetMax, out);
+}
+
+template <int MT, bool FUSED, int RT>
 __global__ void __launch_bounds__(kMaxThreads, 2)
     sherry_decode_kernel(const Params p)
 {
+    static_assert(RT == 1 || RT == 2 || RT == 4, "rows per thread");
     extern __shared__ __align__(16) uint8_t smem[];
     const int M = (int)p.M;
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int64_t r0 = row_begin(p.N, blockIdx.x, p.G), r1 = row_begin(p.N, blockIdx.x + 1, p.G);
     const int Rc = (int)(r1 - r0);
-    const int R = p.R, P = p.P;
+    const int R = p.R, P = p.P, S = p.S;
     const uint32_t s_base = ptx::smem_u32(smem);
     const uint32_t codes_s = s_base + off_codes(M, P, R);
     const int qoff = off_q(M, P, R, p.Kc);
     int8_t* qbuf = reinterpret_cast<int8_t*>(smem + qoff);
-    const int QK = (int)p.Kc * SHERRY_KCHUNK;              // bytes per token row of qbuf
+    const int QK = (int)p.Kc * S;                          // bytes per token row of qbuf
+    int32_t* sums = reinterpret_cast<int32_t*>(smem + off_sums(M, P, R));   // [M][R]
 
     // ---- before the wait: this CTA's codes, alpha, the decode table -------------
     // Row groups start at multiples of 4 rows, so 4 consecutive rows of one word
@@ -181,6 +368,19 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
         for (int ii = tid; ii < Rc; ii += nthr) cp_async4(alpha_s + 4u * (uint32_t)ii, p.alpha + r0 + ii);
         asm volatile("cp.async.commit_group;" ::: "memory");
     }
+    if constexpr (FUSED) {
+        // this CTA's share of the fp32 activations, pulled into L2 while the
+        // previous kernel finishes (a prefetch changes no value)
+        if (tid == 0) {
+            const int64_t bytes = p.M * p.K * 4;
+            const int64_t share = ((bytes + p.G - 1) / p.G + 127) & ~int64_t(127);
+            const int64_t b0 = share * blockIdx.x;
+            if (b0 < bytes)
+                bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.x) + b0,
+                                 (uint32_t)(bytes - b0 < share ? bytes - b0 : share));
+        }
+    }
+    for (int i = tid; i < M * R; i += nthr) sums[i] = 0;
     // the decode table at a 128-byte aligned shared address, so that a lookup
     // address is one LOP3: (code * 4) | table
     const uint32_t table_s = (s_base + kOffTable + 127u) & ~127u;
@@ -188,6 +388,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     ptx::pdl_wait();
 
     // ---- activations -------------------------------------------------------------
+    // qbuf holds token m's K chunk c at byte m * QK + c * S.
     float* scale_s = reinterpret_cast<float*>(smem + kOffScale);
     const int K4 = (int)(p.K >> 2);
     if constexpr (FUSED) {
@@ -198,7 +399,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
         const bool in_regs = K4 <= kXV * nthr;
         for (int m = 0; m < M; ++m) {
             const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)m * p.K);
-            uint32_t* qr = reinterpret_cast<uint32_t*>(qbuf + m * QK);
+            int8_t* qr = qbuf + m * QK;
             float4 v[kXV];
             float mx = 0.0f;
             if (in_regs) {
@@ -231,20 +432,21 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             }
             uint32_t* qo = (p.xq_out && blockIdx.x == 0) ? reinterpret_cast<uint32_t*>(p.xq_out + (int64_t)m * p.K)
                                                           : nullptr;
+            // word idx (activations 4 idx .. 4 idx + 3) sits in chunk idx / 32
             if (in_regs) {
 #pragma unroll
                 for (int u = 0; u < kXV; ++u) {
                     const int idx = tid + u * nthr;
                     if (idx < K4) {
                         const uint32_t w = quant::quantise4(v[u], sc);
-                        qr[idx] = w;
+                        *reinterpret_cast<uint32_t*>(qr + (idx >> 5) * S + 4 * (idx & 31)) = w;
                         if (qo) qo[idx] = w;
                     }
                 }
             } else {
                 for (int i = tid; i < K4; i += nthr) {
                     const uint32_t w = quant::quantise4(xr[i], sc);
-                    qr[i] = w;
+                    *reinterpret_cast<uint32_t*>(qr + (i >> 5) * S + 4 * (i & 31)) = w;
                     if (qo) qo[i] = w;
                 }
             }
@@ -253,16 +455,18 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
         const int K16 = (int)(p.K >> 4);
         for (int m = 0; m < M; ++m)
             for (int i = tid; i < K16; i += nthr)
-                cp_async16(s_base + (uint32_t)(qoff + m * QK + 16 * i), p.xq + (int64_t)m * p.K + 16 * i);
+                cp_async16(s_base + (uint32_t)(qoff + m * QK + (i >> 3) * S + 16 * (i & 7)),
+                           p.xq + (int64_t)m * p.K + 16 * i);
         asm volatile("cp.async.commit_group;" ::: "memory");
         if (tid < M) scale_s[tid] = p.x_scale[tid];
     }
     // zero the activation tail of the last chunk: its padding codes decode to nonzero weights
     {
-        const int tail = QK - (int)p.K;                    // multiple of 32
+        const int used = (int)(p.K - (p.Kc - 1) * SHERRY_KCHUNK);      // bytes of the last chunk in K
+        const int tail = SHERRY_KCHUNK - used;                          // multiple of 32
         for (int i = tid; i < M * tail; i += nthr) {
             const int m = i / tail;
-            qbuf[m * QK + (int)p.K + (i - m * tail)] = 0;
+            qbuf[m * QK + (int)(p.Kc - 1) * S + used + (i - m * tail)] = 0;
         }
     }
     cp_async_wait_all();
@@ -271,61 +475,40 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     // instead of queueing in front of this CTA's activation reads
     ptx::pdl_launch_dependents();
 
-    // ---- decode + dp4a: one row per thread ----------------------------------------
-    // All 32 table loads of a chunk are issued before its dp4a run, which keeps
-    // enough loads in flight with one CTA per SM; the next chunk's code words
-    // are fetched during the current one.
-    const int i = tid % R, part = tid / R;
-    int32_t acc[MT][4];
+    // ---- decode + dp4a: RT rows per thread ----------------------------------------
+    const int qi = tid % p.Q, part = tid / p.Q;
+    int32_t acc[RT][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0;
-    if (part < P && i < Rc) {
-        const uint32_t cbase = codes_s + 4u * (uint32_t)i;
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+    if (part < P && qi * RT < Rc) {
+        const uint32_t cbase = codes_s + 4u * (uint32_t)(qi * RT);
         const uint32_t q_s = s_base + (uint32_t)qoff;
         const int cb = part * p.CPT;
         const int ce = min((int)p.Kc, cb + p.CPT);
-        uint32_t wn[SHERRY_CHUNK_WORDS];
-#pragma unroll
-        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
-            wn[j] = ptx::lds_u32_nv(cbase + 4u * (uint32_t)((cb * SHERRY_CHUNK_WORDS + j) * R));
 #pragma unroll 1
         for (int c = cb; c < ce; ++c) {
-            uint32_t w[SHERRY_CHUNK_WORDS + 1];
+            // the five code words of each of the RT rows: one RT-word load per plane
+            uint32_t w[RT][SHERRY_CHUNK_WORDS + 1];
 #pragma unroll
-            for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) w[j] = wn[j];
-            w[SHERRY_CHUNK_WORDS] = 0;
-            if (c + 1 < ce) {
+            for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) {
+                uint32_t t[RT];
+                lds_vec<RT>(cbase + 4u * (uint32_t)((c * SHERRY_CHUNK_WORDS + j) * R), t);
 #pragma unroll
-                for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
-                    wn[j] = ptx::lds_u32_nv(cbase + 4u * (uint32_t)(((c + 1) * SHERRY_CHUNK_WORDS + j) * R));
+                for (int r = 0; r < RT; ++r) w[r][j] = t[r];
             }
-            // table entries of the chunk's 32 codes
-            uint32_t e[32];
 #pragma unroll
-            for (int g = 0; g < 32; ++g) {
-                // byte offset of group g's code in the table: (bits [5g, 5g+5)) * 4
-                const int bit = 5 * g, wi = bit >> 5, off = bit & 31;
-                uint32_t v;
-                if (off == 0) v = w[wi] << 2;
-                else if (off == 1) v = w[wi] << 1;
-                else if (off <= 27) v = w[wi] >> (off - 2);
-                else v = __funnelshift_r(w[wi], w[wi + 1], off - 2);
-                e[g] = ptx::lds_u32_nv((v & 0x7Cu) | table_s);
-            }
-            const uint32_t qc = q_s + (uint32_t)(c * SHERRY_KCHUNK);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                if (m >= M) break;
-#pragma unroll
-                for (int g4 = 0; g4 < 8; ++g4) {
-                    uint32_t qv[4];
-                    lds_vec<4>(qc + (uint32_t)(m * QK + 16 * g4), qv);
-                    acc[m][0] = __dp4a((int)e[4 * g4 + 0], (int)qv[0], acc[m][0]);
-                    acc[m][1] = __dp4a((int)e[4 * g4 + 1], (int)qv[1], acc[m][1]);
-                    acc[m][2] = __dp4a((int)e[4 * g4 + 2], (int)qv[2], acc[m][2]);
-                    acc[m][3] = __dp4a((int)e[4 * g4 + 3], (int)qv[3], acc[m][3]);
-                }
-            }
+            for (int r = 0; r < RT; ++r) w[r][SHERRY_CHUNK_WORDS] = 0;
+            const uint32_t qc = q_s + (uint32_t)(c * S);
+            piece<0, MT, RT>(w, table_s, qc, QK, M, acc);
+            piece<1, MT, RT>(w, table_s, qc, QK, M, acc);
+            piece<2, MT, RT>(w, table_s, qc, QK, M, acc);
+            piece<3, MT, RT>(w, table_s, qc, QK, M, acc);
+            piece<4, MT, RT>(w, table_s, qc, QK, M, acc);
+            piece<5, MT, RT>(w, table_s, qc, QK, M, acc);
+            piece<6, MT, RT>(w, table_s, qc, QK, M, acc);
+            piece<7, MT, RT>(w, table_s, qc, QK, M, acc);
         }
     }
 
@@ -335,13 +518,28 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     if (part < P) {
 #pragma unroll
         for (int m = 0; m < MT; ++m)
-            if (m < M) red[(part * M + m) * R + i] = (acc[m][0] + acc[m][1]) + (acc[m][2] + acc[m][3]);
+            if (m < M)
+#pragma unroll
+                for (int r = 0; r < RT; ++r) red[(part * M + m) * R + qi * RT + r] = acc[r][m];
     }
     __syncthreads();
-    for (int idx = tid; idx < M * Rc; idx += nthr) {
+    // output o = (token m, row i): T threads share its P parts, each adding
+    // its share into the row total with a shared atomic
+    const int O = M * Rc;
+    if (O > 0) {
+        const int T = O >= nthr ? 1 : nthr / O;
+        for (int idx = tid; idx < O * T; idx += nthr) {
+            const int o = idx % O, s = idx / O;
+            const int m = o / Rc, ii = o - m * Rc;
+            int32_t v = 0;
+            for (int pp = s; pp < P; pp += T) v += red[(pp * M + m) * R + ii];
+            atomicAdd(&sums[m * R + ii], v);
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < O; idx += nthr) {
         const int m = idx / Rc, ii = idx - m * Rc;
-        int32_t a32 = 0;
-        for (int pp = 0; pp < P; ++pp) a32 += red[(pp * M + m) * R + ii];
+        const int32_t a32 = sums[m * R + ii];
         const int64_t n = r0 + ii;
         if (p.acc) p.acc[m * p.N + n] = a32;
         if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, alpha_sm[ii]), scale_s[m]);

@@ -63,6 +63,28 @@ __global__ void __launch_bounds__(kQuantThreads)
 }
 
 // ---------------------------------------------------------------------------
+// Self-test of failure detection: one warp initialises an mbarrier that
+// nothing ever arrives on and waits for its first phase with the bounded
+// wait every kernel of the library uses.  When the bound runs out it records
+// SHERRY_DEV_TIMEOUT_SELFTEST in the device status word and returns.  No
+// bulk copy and no tensor memory is involved, so nothing is in flight when
+// the wait gives up.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) wait_selftest_kernel(uint64_t limit_ns, unsigned* status)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = ptx::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(b, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncwarp();
+    const bool done = ptx::mbar_wait_bounded(b, 0, limit_ns);
+    if (!__all_sync(0xffffffffu, done) && threadIdx.x == 0)
+        atomicCAS(status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_SELFTEST);
+}
+
+// ---------------------------------------------------------------------------
 // Repack: canonical stream -> kernel-native layout (one thread per word).
 // ---------------------------------------------------------------------------
 __global__ void repack_kernel(const uint8_t* __restrict__ codes, int64_t N, int64_t K, uint32_t* __restrict__ out,
@@ -248,30 +270,29 @@ int64_t tc_grid(int64_t T, int64_t U, int64_t sms, int64_t Kc, int bn)
     return std::min<int64_t>(g, U);
 }
 
-int get_workspace(size_t bytes, cudaStream_t stream, void** out)
+// The per-device split-K workspace set aside by sherry_reserve: never
+// allocated here (the asynchronous entry points allocate nothing and never
+// synchronise); SHERRY_ERR_WORKSPACE when it is smaller than a call needs.
+int get_workspace(size_t bytes, void** out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SHERRY_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mutex);
-    if ((int)g_ws.size() <= dev) g_ws.resize(dev + 1);
-    Workspace& w = g_ws[dev];
-    if (w.bytes < bytes) {
-        if (w.ptr) {
-            if (cudaStreamSynchronize(stream) != cudaSuccess) return SHERRY_ERR_CUDA;
-            cudaFree(w.ptr);
-            w.ptr = nullptr;
-            w.bytes = 0;
-        }
-        size_t nb = std::max<size_t>(bytes, size_t(1) << 20);
-        if (cudaMalloc(&w.ptr, nb) != cudaSuccess) {
-            w.ptr = nullptr;
-            return SHERRY_ERR_CUDA;
-        }
-        if (cudaMemsetAsync(w.ptr, 0, nb, stream) != cudaSuccess) return SHERRY_ERR_CUDA;
-        w.bytes = nb;
-    }
-    *out = w.ptr;
+    if ((int)g_ws.size() <= dev || g_ws[dev].bytes < bytes) return SHERRY_ERR_WORKSPACE;
+    *out = g_ws[dev].ptr;
     return SHERRY_OK;
+}
+
+// Token tile of the tensor-core kernel for M tokens (the dispatch of
+// sherry_gemm_tc and sherry_w4a8_gemm_tc).
+int tc_token_tile(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M < 1536 ? 128 : 192; }
+
+// Split-K workspace for every launch of up to M tokens on `sms` SMs: the
+// partial-sum slots of at most one CTA per SM, BN tokens x 128 rows each, and
+// one arrival counter per CTA.
+size_t tc_workspace_bytes(int64_t M, int sms)
+{
+    return (size_t)sms * tc_token_tile(M) * SHERRY_TILE_ROWS * sizeof(int32_t) + (size_t)sms * sizeof(uint32_t);
 }
 
 // fp32 y [M][N]: boxes of 32 rows n x box_m tokens m (no swizzle), one per
@@ -354,12 +375,18 @@ int launch_tc(const int8_t* x, const float* xs, const void* wn, const float* alp
     p.Kc = sherry_k_chunks(K);
     p.U = p.TM * p.TN * p.Kc;
     const int64_t grid = tc_grid(p.TM * p.TN, p.U, di.sms, p.Kc, BN);
-    void* ws = nullptr;
-    const size_t ws_acc = (size_t)grid * BN * SHERRY_TILE_ROWS * sizeof(int32_t);
-    st = get_workspace(ws_acc + (size_t)grid * sizeof(uint32_t), stream, &ws);
-    if (st != SHERRY_OK) return st;
-    p.ws = static_cast<int32_t*>(ws);
-    p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ws_acc);
+    // the workspace is touched only by tiles whose K range is split across
+    // CTAs: the last T mod G tiles (none when every CTA takes whole tiles)
+    p.ws = nullptr;
+    p.counters = nullptr;
+    if ((p.TM * p.TN) % grid != 0) {
+        void* ws = nullptr;
+        const size_t ws_acc = (size_t)grid * BN * SHERRY_TILE_ROWS * sizeof(int32_t);
+        st = get_workspace(ws_acc + (size_t)grid * sizeof(uint32_t), &ws);
+        if (st != SHERRY_OK) return st;
+        p.ws = static_cast<int32_t*>(ws);
+        p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ws_acc);
+    }
     p.status = device_status_ptr();
     if (!p.status) return SHERRY_ERR_CUDA;
 
@@ -463,44 +490,27 @@ int launch_gemv(const int8_t* x, const float* xs, const void* wn, const float* a
     return cuda_status(cudaLaunchKernelEx(&cfg, gemv::sherry_gemv_kernel<MT>, p));
 }
 
-// Work split of the decode kernel: G CTAs of at most R rows (one per SM
-// unless the codes of R rows would not fit the shared-memory budget), P
-// K-parts of CPT chunks per row, R * P <= kMaxThreads.  False if even one
-// row does not fit.
-struct DecodePlan {
-    int G, R, P, CPT, threads, smem;
-};
-
-bool decode_plan(int64_t N, int64_t Kc, int64_t M, int sms, DecodePlan* out)
+template <int MT, bool FUSED, int RT>
+int launch_decode_rt(const decode::Params& p, const decode::Plan& pl, cudaStream_t stream)
 {
-    // at least 4 rows per CTA: row boundaries rounded to 4 rows then leave no CTA empty
-    const int64_t gmax = std::max<int64_t>(1, N / 4);
-    int64_t G = std::min<int64_t>(sms, gmax);
-    for (int iter = 0; iter < 64; ++iter) {
-        const int64_t R = ((N + G - 1) / G + 3 + 3) & ~int64_t(3);     // rounded groups, a multiple of 4
-        const int64_t RQ = R;
-        if (RQ > decode::kMaxThreads) {
-            G = std::min<int64_t>(gmax, (N + decode::kMaxThreads - 1) / decode::kMaxThreads);
-            continue;
-        }
-        int64_t P = std::max<int64_t>(1, std::min<int64_t>(Kc, decode::kMaxThreads / RQ));
-        const int64_t CPT = (Kc + P - 1) / P;
-        P = (Kc + CPT - 1) / CPT;
-        const int64_t smem = decode::smem_bytes((int)M, (int)P, (int)R, Kc);
-        if (smem <= decode::kSmemBudget) {
-            if (G > 0x7fffffff) return false;
-            out->G = (int)G;
-            out->R = (int)R;
-            out->P = (int)P;
-            out->CPT = (int)CPT;
-            out->threads = (int)std::max<int64_t>(32, (RQ * P + 31) / 32 * 32);
-            out->smem = (int)smem;
-            return true;
-        }
-        if (R <= 4 || G >= gmax) return false;
-        G = std::min<int64_t>(gmax, (N + R / 2 - 1) / (R / 2));       // halve the rows per CTA
-    }
-    return false;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    // One shared-memory carveout for every shape: left to the driver, the
+    // L1/shared split follows each launch's request, and consecutive layers
+    // of different shapes (27, 70 and 88 KB) then cannot share an SM, so the
+    // next layer's CTAs lose their early start (measured: 11.2 us per call
+    // alternating two shapes that take 7.6 and 9.0 us on their own).
+    std::call_once(attr_once, [&] {
+        attr_err = cudaFuncSetAttribute(decode::sherry_decode_kernel<MT, FUSED, RT>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, decode::kSmemBudgetMax);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(decode::sherry_decode_kernel<MT, FUSED, RT>,
+                                            cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            cudaSharedmemCarveoutMaxShared);
+    });
+    if (attr_err != cudaSuccess) return SHERRY_ERR_CUDA;
+    return cuda_status(launch_pdl(decode::sherry_decode_kernel<MT, FUSED, RT>, dim3((unsigned)pl.G),
+                                  dim3((unsigned)pl.threads), (size_t)pl.smem, stream, p));
 }
 
 template <int MT, bool FUSED>
@@ -512,59 +522,59 @@ int launch_decode(const decode::Params& p0, cudaStream_t stream)
     decode::Params p = p0;
     p.Kc = sherry_k_chunks(p.K);
     if (p.M > MT) return SHERRY_ERR_UNSUPPORTED_SHAPE;
-    DecodePlan pl;
-    if (!decode_plan(p.N, p.Kc, p.M, di.sms, &pl)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    decode::Plan pl;
+    if (!decode::plan(p.N, p.Kc, p.M, di.sms, &pl)) return SHERRY_ERR_UNSUPPORTED_SHAPE;
     p.G = pl.G;
     p.R = pl.R;
+    p.Q = pl.Q;
     p.P = pl.P;
     p.CPT = pl.CPT;
+    p.S = pl.S;
     if (pl.smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    // One shared-memory carveout for every shape: left to the driver, the
-    // L1/shared split follows each launch's request, and consecutive layers
-    // of different shapes (27, 70 and 88 KB) then cannot share an SM, so the
-    // next layer's CTAs lose their early start (measured: 11.2 us per call
-    // alternating two shapes that take 7.6 and 9.0 us on their own).
-    std::call_once(attr_once, [&] {
-        attr_err = cudaFuncSetAttribute(decode::sherry_decode_kernel<MT, FUSED>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, decode::kSmemBudget);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(decode::sherry_decode_kernel<MT, FUSED>,
-                                            cudaFuncAttributePreferredSharedMemoryCarveout,
-                                            cudaSharedmemCarveoutMaxShared);
-    });
-    if (attr_err != cudaSuccess) return SHERRY_ERR_CUDA;
-    return cuda_status(launch_pdl(decode::sherry_decode_kernel<MT, FUSED>, dim3((unsigned)pl.G),
-                                  dim3((unsigned)pl.threads), (size_t)pl.smem, stream, p));
+    if (pl.RT == 4) {
+        if constexpr (MT <= 2) return launch_decode_rt<MT, FUSED, 4>(p, pl, stream);
+        else return SHERRY_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (pl.RT == 2) return launch_decode_rt<MT, FUSED, 2>(p, pl, stream);
+    return launch_decode_rt<MT, FUSED, 1>(p, pl, stream);
 }
 
 // Per-device buffer for the int8 activations and scales of sherry_linear
-// when the caller passes none and the fused kernel does not apply.
+// when the caller passes none and the fused kernel does not apply; set aside
+// by sherry_reserve, never allocated here.
 std::vector<Workspace> g_act;
 
-int get_act_buffer(size_t bytes, cudaStream_t stream, void** out)
+size_t act_buffer_bytes(int64_t M, int64_t K) { return (((size_t)M * (size_t)K + 255) & ~size_t(255)) + 4 * (size_t)M; }
+
+int get_act_buffer(size_t bytes, void** out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SHERRY_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mutex);
-    if ((int)g_act.size() <= dev) g_act.resize(dev + 1);
-    Workspace& w = g_act[dev];
-    if (w.bytes < bytes) {
-        if (w.ptr) {
-            if (cudaStreamSynchronize(stream) != cudaSuccess) return SHERRY_ERR_CUDA;
-            cudaFree(w.ptr);
-            w.ptr = nullptr;
-            w.bytes = 0;
-        }
-        size_t nb = std::max<size_t>(bytes, size_t(1) << 20);
-        if (cudaMalloc(&w.ptr, nb) != cudaSuccess) {
-            w.ptr = nullptr;
-            return SHERRY_ERR_CUDA;
-        }
-        w.bytes = nb;
+    if ((int)g_act.size() <= dev || g_act[dev].bytes < bytes) return SHERRY_ERR_WORKSPACE;
+    *out = g_act[dev].ptr;
+    return SHERRY_OK;
+}
+
+// Grow one per-device buffer to at least `bytes` (host-synchronous; the
+// device is idle before an older, smaller buffer is freed), zero-filled.
+int grow_buffer(Workspace& w, size_t bytes)
+{
+    if (w.bytes >= bytes) return SHERRY_OK;
+    if (w.ptr) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return SHERRY_ERR_CUDA;
+        cudaFree(w.ptr);
+        w.ptr = nullptr;
+        w.bytes = 0;
     }
-    *out = w.ptr;
+    void* ptr = nullptr;
+    if (cudaMalloc(&ptr, bytes) != cudaSuccess) return SHERRY_ERR_CUDA;
+    if (cudaMemset(ptr, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        cudaFree(ptr);
+        return SHERRY_ERR_CUDA;
+    }
+    w.ptr = ptr;
+    w.bytes = bytes;
     return SHERRY_OK;
 }
 
@@ -767,8 +777,8 @@ int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnativ
         DeviceInfo di;
         st = device_info(&di);
         if (st != SHERRY_OK) return st;
-        DecodePlan pl;
-        if (decode_plan(N, sherry_k_chunks(K), M, di.sms, &pl))
+        decode::Plan pl;
+        if (decode::plan(N, sherry_k_chunks(K), M, di.sms, &pl))
             return sherry_gemm_decode(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
     }
     return sherry_gemm_tc(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
@@ -810,8 +820,8 @@ int sherry_linear_ex(const float* x, const void* Wnative, const float* alpha, fl
         DeviceInfo di;
         int st = device_info(&di);
         if (st != SHERRY_OK) return st;
-        DecodePlan pl;
-        if (decode_plan(N, sherry_k_chunks(K), M, di.sms, &pl)) {
+        decode::Plan pl;
+        if (decode::plan(N, sherry_k_chunks(K), M, di.sms, &pl)) {
             decode::Params p = {};
             p.wnative = static_cast<const uint8_t*>(Wnative);
             p.x = x;
@@ -823,14 +833,16 @@ int sherry_linear_ex(const float* x, const void* Wnative, const float* alpha, fl
             p.M = M;
             p.N = N;
             p.K = K;
-            static_assert(SHERRY_LINEAR_FUSED_MAX_M == 1, "fused launches instantiated for one token");
-            return launch_decode<1, true>(p, s);
+            static_assert(SHERRY_LINEAR_FUSED_MAX_M <= 4, "fused launches instantiated for up to 4 tokens");
+            if (M == 1) return launch_decode<1, true>(p, s);
+            if (M == 2) return launch_decode<2, true>(p, s);
+            return launch_decode<4, true>(p, s);
         }
     }
     if (!x_i8) {
         void* buf = nullptr;
         const size_t qbytes = ((size_t)M * (size_t)K + 255) & ~size_t(255);
-        int st = get_act_buffer(qbytes + (size_t)M * sizeof(float), s, &buf);
+        int st = get_act_buffer(act_buffer_bytes(M, K), &buf);
         if (st != SHERRY_OK) return st;
         x_i8 = static_cast<int8_t*>(buf);
         x_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(buf) + qbytes);
@@ -912,12 +924,48 @@ int sherry_gemm_noalloc(const int8_t* x_i8, const float* x_scale, const void* Wn
         DeviceInfo di;
         st = device_info(&di);
         if (st != SHERRY_OK) return st;
-        DecodePlan pl;
-        if (decode_plan(N, sherry_k_chunks(K), M, di.sms, &pl))
+        decode::Plan pl;
+        if (decode::plan(N, sherry_k_chunks(K), M, di.sms, &pl))
             return sherry_gemm_decode(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, stream);
     }
     if (M <= 16) return launch_tc_noalloc<16, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
     return launch_tc_noalloc<32, 4>(x_i8, x_scale, Wnative, alpha, y, acc, M, N, K, s);
+}
+
+int sherry_selftest_wait(uint64_t limit_ns, void* stream)
+{
+    if (limit_ns == 0 || limit_ns > 1000000000ull) return SHERRY_ERR_INVALID_ARG;
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != SHERRY_OK) return st;
+    unsigned* status = device_status_ptr();
+    if (!status) return SHERRY_ERR_CUDA;
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, status);
+    return cuda_status(cudaGetLastError());
+}
+
+size_t sherry_workspace_bytes(int64_t max_M, int64_t max_K)
+{
+    if (max_M < 1 || max_K < 1) return 0;
+    DeviceInfo di;
+    if (device_info(&di) != SHERRY_OK) return 0;
+    return tc_workspace_bytes(max_M, di.sms) + act_buffer_bytes(max_M, max_K);
+}
+
+int sherry_reserve(int64_t max_M, int64_t max_K)
+{
+    if (max_M < 1 || max_K < 1 || max_M > SHERRY_MAX_DIM || max_K > SHERRY_MAX_K) return SHERRY_ERR_INVALID_ARG;
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != SHERRY_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SHERRY_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((int)g_ws.size() <= dev) g_ws.resize(dev + 1);
+    if ((int)g_act.size() <= dev) g_act.resize(dev + 1);
+    st = grow_buffer(g_ws[dev], tc_workspace_bytes(max_M, di.sms));
+    if (st != SHERRY_OK) return st;
+    return grow_buffer(g_act[dev], act_buffer_bytes(max_M, max_K));
 }
 
 int sherry_last_device_status(int reset)
@@ -925,6 +973,17 @@ int sherry_last_device_status(int reset)
     unsigned v = 0;
     if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return -1;
     if (reset) {
+        // A launch whose bounded wait ran out may have left split-K partial
+        // sums and arrival counters behind: the workspace of this device is
+        // zeroed again before the next call can use it.
+        if (v != 0) {
+            int dev = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return -1;
+            std::lock_guard<std::mutex> lk(g_mutex);
+            if ((int)g_ws.size() > dev && g_ws[dev].ptr &&
+                (cudaMemset(g_ws[dev].ptr, 0, g_ws[dev].bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess))
+                return -1;
+        }
         unsigned z = 0;
         if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(z)) != cudaSuccess) return -1;
     }

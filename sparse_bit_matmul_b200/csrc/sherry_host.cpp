@@ -65,6 +65,7 @@ const char* sherry_status_string(int status)
     case SHERRY_ERR_NONFINITE: return "non-finite weight";
     case SHERRY_ERR_CUDA: return "CUDA error";
     case SHERRY_ERR_DEVICE: return "unsupported device";
+    case SHERRY_ERR_WORKSPACE: return "workspace too small: call sherry_reserve first";
     default: return "unknown status";
     }
 }

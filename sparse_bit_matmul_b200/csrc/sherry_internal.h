@@ -95,4 +95,5 @@ enum sherry_device_code : unsigned {
     SHERRY_DEV_TIMEOUT_EPILOGUE = 0x104,
     SHERRY_DEV_TIMEOUT_DRAIN = 0x105,
     SHERRY_DEV_TMEM_ALLOC = 0x106,
+    SHERRY_DEV_TIMEOUT_SELFTEST = 0x107,
 };

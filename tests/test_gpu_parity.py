@@ -172,30 +172,34 @@ def test_gemm_zero_token_and_repeat():
 
 # ----------------------------------------------- full-size configurations
 def _full_size_check(cfg, copy, M_list, K, N, int_mm=True, kernels=("auto",)):
+    """One workload configuration at full size.  The codes and alpha of every
+    row are compared with the oracle's.  For M <= 16 the oracle computes
+    every output, and the whole int32 acc (bit-exact) and y (1e-6 relative)
+    are compared.  Larger M compares oracle rows sampled at tile edges and at
+    random, and every accumulator against torch._int_mm over the oracle's
+    ternary weights."""
     W = synth.config_weights(cfg, copy, K, N)
     native, alpha_d, codes, alpha = upload_weights(W)
+    T_full, a_full = oracle.quantise(W)
+    assert np.array_equal(codes, oracle.pack(T_full))
+    assert np.array_equal(alpha, a_full)
     rows = rows_sample(N, seed=cfg * 7 + N)
-    T_rows, a_rows = oracle.quantise(W[rows])
-    assert np.array_equal(codes[rows], oracle.pack(T_rows))
-    assert np.array_equal(alpha[rows], a_rows)
-    T_full = None
     for M in M_list:
         x = synth.config_activations(cfg, copy, M, K)
         q_o, s_o = oracle.quant_act(x)
-        acc_o = oracle.gemm(q_o, T_rows)
+        cols = np.arange(N) if M <= 16 else rows
+        acc_o = oracle.gemm(q_o, T_full if M <= 16 else T_full[rows])
+        y_o = oracle.epilogue(acc_o, a_full[cols], s_o)
         for kern in kernels:
             if not _kernel_serves(kern, M, K):
                 continue
             y, acc, q, s = run_gpu(x, native, alpha_d, N, kern)
             assert np.array_equal(q, q_o) and np.array_equal(s, s_o)
-            assert np.array_equal(acc[:, rows], acc_o), kern
-            y_ref_rows = oracle.epilogue(acc_o, a_rows, s_o)
-            assert_y_close(y[:, rows], y_ref_rows)
+            assert np.array_equal(acc[:, cols], acc_o), kern
+            assert_y_close(y[:, cols], y_o)
             y2, _, _, _ = run_gpu(x, native, alpha_d, N, kern, with_acc=False)
             assert np.array_equal(y2, y), kern          # y-only path (TMA stores) gives the same y
         if int_mm and M > 16:
-            if T_full is None:
-                T_full, _ = oracle.quantise(W)
             ref = torch._int_mm(torch.from_numpy(q_o).cuda(), torch.from_numpy(T_full).cuda().t().contiguous())
             assert torch.equal(torch.from_numpy(acc).cuda(), ref)
     return W
@@ -203,12 +207,12 @@ def _full_size_check(cfg, copy, M_list, K, N, int_mm=True, kernels=("auto",)):
 
 @pytest.mark.parametrize("K,N", synth.PROJ_SHAPES)
 def test_config1_decode_full_size(K, N):
-    _full_size_check(1, 0, [1], K, N, kernels=("auto", "linear", "tc", "gemv"))
+    _full_size_check(1, 0, [1], K, N, kernels=("auto", "linear", "decode", "tc", "gemv"))
 
 
 @pytest.mark.parametrize("K,N", synth.PROJ_SHAPES)
 def test_config2_small_batch_full_size(K, N):
-    _full_size_check(2, 0, [4, 8, 16, 32], K, N, kernels=("auto", "linear", "tc"))
+    _full_size_check(2, 0, [4, 8, 16, 32], K, N, kernels=("auto", "linear", "decode", "tc"))
 
 
 @pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096)])
@@ -217,9 +221,39 @@ def test_config3_prefill_full_size(K, N):
 
 
 def test_config4_heavy_tail_full_size():
-    W = _full_size_check(4, 0, [1, 128, 4096], 8192, 28672, kernels=("auto", "linear", "tc"))
+    W = _full_size_check(4, 0, [1, 128, 4096], 8192, 28672, kernels=("auto", "linear", "decode", "tc"))
     T, _ = oracle.quantise(W)
     assert np.all(np.count_nonzero(T.reshape(28672, -1, 4), axis=2) == 3)
+
+
+@pytest.mark.parametrize("M,N,K,kernel", [(1, 256, 14336, "decode"), (2, 256, 14336, "decode"),
+                                          (1, 256, 14336, "linear"), (1, 256, 14336, "gemv"),
+                                          (4, 256, 14336, "tc"), (16, 256, 14336, "tc"),
+                                          (4, 256, 14336, "gemv"), (8, 256, 4096, "decode"),
+                                          (130, 512, 14336, "tc")])
+def test_accumulator_extremes(M, N, K, kernel):
+    """The largest sums the method can form: every activation quantises to
+    +127 or -127 and every row is all +1 or all -1 on its kept weights, so
+    |acc| = 127 * 0.75 K (1,365,504 at K = 14336).  Through the decode
+    kernel, the fused linear path, the table GEMV and the tensor cores (the
+    small-M shapes split every tile's K range over many CTAs, whose int32
+    partial sums meet in the workspace)."""
+    # groups of 4 positive weights with distinct magnitudes: position 0 is
+    # zeroed, 1..3 keep +1; the second half of the rows is negated
+    g = np.array([1.0, 2.0, 3.0, 4.0], dtype=np.float32) * 0.01
+    W = np.tile(g, (N, K // 4))
+    W[N // 2:] *= -1.0
+    x = np.ones((M, K), dtype=np.float32)
+    x[1::2] *= -1.0                                     # odd tokens: every activation -127
+    y_o, acc_o, q_o, s_o, codes_o, alpha_o = oracle.reference(x, W)
+    assert np.all(np.abs(q_o) == 127)
+    full = 127 * 3 * (K // 4)
+    assert np.all(np.abs(acc_o) == full)
+    native, alpha_d, codes, alpha = upload_weights(W)
+    assert np.array_equal(codes, codes_o)
+    y, acc, q, s = run_gpu(x, native, alpha_d, N, kernel)
+    assert np.array_equal(acc, acc_o)
+    assert_y_close(y, y_o)
 
 
 def test_config0_tiny_exact():

@@ -106,3 +106,61 @@ def test_pack_thread_count_independent(lib):
         env = dict(os.environ, OMP_NUM_THREADS=nt)
         outs.append(subprocess.check_output([sys.executable, "-c", code], env=env, cwd=ROOT).strip())
     assert outs[0] == outs[1]
+
+
+def _function_spans(text):
+    """(name, start, end) of every function body in a C/C++/CUDA source:
+    the identifier before the parameter list of each '{' that opens a
+    function, matched to its closing brace."""
+    spans = []
+    for m in re.finditer(r"\b([A-Za-z_]\w*)\s*\(([^;{}()]|\([^;{}()]*\))*\)\s*(const\s*)?\{", text):
+        name = m.group(1)
+        if name in ("if", "for", "while", "switch", "catch", "sizeof", "return"):
+            continue
+        depth, i = 0, m.end() - 1
+        while i < len(text):
+            if text[i] == "{":
+                depth += 1
+            elif text[i] == "}":
+                depth -= 1
+                if depth == 0:
+                    break
+            i += 1
+        spans.append((name, m.start(), i))
+    return spans
+
+
+def test_async_entry_points_never_allocate_or_synchronise():
+    """Allocation, freeing and host synchronisation appear in the device
+    source only inside the host-synchronous entry points (sherry_reserve and
+    its buffer growth, the status read with its reset); the per-call
+    scratch clearing of sherry_gemm_noalloc is the only stream-ordered
+    memset.  So none of the asynchronous entry points can reach them."""
+    path = os.path.join(ROOT, "sparse_bit_matmul_b200", "csrc", "sherry_cuda.cu")
+    text = open(path).read()
+    text = re.sub(r"//[^\n]*", "", re.sub(r"/\*.*?\*/", "", text, flags=re.S))
+    spans = _function_spans(text)
+    allowed = {
+        "cudaMalloc": {"grow_buffer"},
+        "cudaFree": {"grow_buffer"},
+        "cudaDeviceSynchronize": {"grow_buffer", "sherry_last_device_status"},
+        "cudaStreamSynchronize": set(),
+        "cudaMemset": {"grow_buffer", "sherry_last_device_status"},
+        "cudaMemsetAsync": {"launch_tc_noalloc"},
+        "cudaMallocAsync": set(),
+        "cudaMallocManaged": set(),
+    }
+    callers = {"grow_buffer": {"sherry_reserve"}}
+    for call, ok in allowed.items():
+        for m in re.finditer(r"\b" + call + r"\s*\(", text):
+            inner = [sp for sp in spans if sp[1] <= m.start() <= sp[2]]
+            assert inner, f"{call} outside any function"
+            name = min(inner, key=lambda sp: sp[2] - sp[1])[0]
+            assert name in ok, f"{call} called in {name}"
+    # grow_buffer itself is reached only from sherry_reserve
+    for m in re.finditer(r"\bgrow_buffer\s*\(", text):
+        inner = [sp for sp in spans if sp[1] <= m.start() <= sp[2] and sp[0] != "grow_buffer"]
+        if not inner:
+            continue                                   # its own definition
+        name = min(inner, key=lambda sp: sp[2] - sp[1])[0]
+        assert name in callers["grow_buffer"], f"grow_buffer called in {name}"
