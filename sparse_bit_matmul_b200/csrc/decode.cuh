@@ -15,9 +15,7 @@
 //     global memory, no workspace, no clusters.
 //   * Before griddepcontrol.wait the CTA streams its rows' codes (the rotated
 //     word planes of the native layout) into shared memory with 16-byte
-//     cp.async copies, and asks L2 to prefetch its share of the fp32
-//     activations (a prefetch has no effect on values, so it may run before
-//     the previous kernel has finished writing them).  Weights never depend
+//     cp.async copies.  Weights never depend
 //     on the previous kernel, so their fetch overlaps its decode.  The CTA
 //     lets the next kernel start only once its own activations are in
 //     shared memory, so that the next kernel's weight stream does not queue
@@ -38,9 +36,8 @@
 //     broadcasts.  Activation chunks sit S >= 128 bytes apart, S chosen on
 //     the host so that the few K-parts that share a warp read different
 //     banks.
-//   * The K-parts of a row are summed in shared memory (every thread adds a
-//     share of the parts into the row's total with a shared atomic), and the
-//     epilogue writes y (and acc) with coalesced stores.
+//   * The K-parts of a row are summed in shared memory and the epilogue writes
+//     y (and acc) with coalesced stores.
 #pragma once
 
 #include <cstdint>
@@ -73,28 +70,28 @@ struct Params {
     int R;                       // largest row count of a CTA, a multiple of 4
     int Q;                       // row groups of RT rows: R / RT
     int P;                       // K-parts per row
-    int CPT;                     // chunks per K-part
+    int CPT;                     // chunks per K-part: the loop steps; step k covers chunk p * CPT + k of part p
+    int NS;                      // ring slots of code steps held in shared memory (NS >= CPT: all of them)
     int S;                       // bytes between consecutive K chunks of the int8 activation buffer
 };
 
 // Shared memory: table | scales | warp maxima (two token slots) | partial sums [P][M][R] |
-// row totals [M][R] | alpha [R] | codes [Kc][5][R] words | activations [M][Kc][S] int8.
+// alpha [R] | code ring [NS][P][5][R] words | activations [M][Kc][S] int8.
 constexpr int kOffTable = 0;                              // 32 x u32, 128-byte aligned inside 256 bytes
 constexpr int kOffScale = 256;                            // [kMaxM] f32 s
 constexpr int kOffWarpMax = kOffScale + kMaxM * 4;        // [2][16 warps] f32
 constexpr int kOffRed = kOffWarpMax + 2 * 16 * 4;
 static_assert(kMaxThreads / 32 <= 16, "warp-maximum slots");
 static_assert(kOffRed % 16 == 0, "alignment");
-__host__ __device__ inline int off_sums(int M, int P, int R) { return (kOffRed + P * M * R * 4 + 15) & ~15; }
-__host__ __device__ inline int off_alpha(int M, int P, int R) { return (off_sums(M, P, R) + M * R * 4 + 15) & ~15; }
+__host__ __device__ inline int off_alpha(int M, int P, int R) { return (kOffRed + P * M * R * 4 + 15) & ~15; }
 __host__ __device__ inline int off_codes(int M, int P, int R) { return (off_alpha(M, P, R) + R * 4 + 15) & ~15; }
-__host__ __device__ inline int off_q(int M, int P, int R, int64_t Kc)
+__host__ __device__ inline int off_q(int M, int P, int R, int NS)
 {
-    return (off_codes(M, P, R) + (int)Kc * SHERRY_CHUNK_WORDS * R * 4 + 15) & ~15;
+    return (off_codes(M, P, R) + NS * P * SHERRY_CHUNK_WORDS * R * 4 + 15) & ~15;
 }
-__host__ __device__ inline int smem_bytes(int M, int P, int R, int64_t Kc, int S)
+__host__ __device__ inline int smem_bytes(int M, int P, int R, int NS, int64_t Kc, int S)
 {
-    return off_q(M, P, R, Kc) + M * (int)Kc * S;
+    return off_q(M, P, R, NS) + M * (int)Kc * S;
 }
 
 __device__ __forceinline__ uint32_t expand_code(uint32_t c)
@@ -126,11 +123,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// L2 prefetch of a byte range (16-byte aligned start, size a multiple of 16)
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 
 // N consecutive 32-bit words from a shared address (aligned to 4 N bytes).
 template <int N>
@@ -207,21 +199,30 @@ inline int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 inline int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 inline int min_i(int a, int b) { return a < b ? a : b; }
 
-// Work split of the decode kernel: G CTAs of at most R rows (one per SM
-// unless the codes of R rows would not fit the shared-memory budget), row
-// groups of RT rows (Q = R / RT of them), P K-parts of CPT chunks per row,
-// Q * P <= kMaxThreads.  RT is the largest that the token count's registers
-// allow and that still gives the CTA at least kMinBusyThreads working
-// threads.  False if even one row does not fit.
+// Work split of the decode kernel: G CTAs of at most R rows, row groups of
+// RT rows (Q = R / RT of them), P K-parts of CPT chunks per row, Q * P <=
+// kMaxThreads.  RT is the largest that the token count's registers allow and
+// that still gives the CTA at least kMinBusyThreads working threads.  The
+// codes live in a ring of NS loop steps (step k holds chunk p * CPT + k of
+// every part p for all R rows): when every step fits (NS = CPT), all of a
+// CTA's codes are fetched before the dependency wait, overlapping the
+// previous kernel; otherwise the CTA streams them, fetching step k + NS while
+// it decodes step k, and the grid takes two CTAs per SM so that the decode
+// runs with twice the warps.
 struct Plan {
-    int G, R, RT, Q, P, CPT, threads, smem, S;
+    int G, R, RT, Q, P, CPT, NS, threads, smem, S;
 };
 
 constexpr int kMinBusyThreads = 320;
+constexpr int kMaxRing = 4;                 // ring slots when the codes stream
 
 // Rows per thread that the registers allow for MT tokens: RT x MT
 // accumulators plus RT x 5 code words and RT x 4 table entries live at once.
 inline int rt_max(int64_t M) { return M <= 2 ? 4 : 2; }
+// Rows per thread tried first: one token takes one row per thread (its loop
+// keeps a whole chunk's table loads in flight; measured faster live than
+// several rows per thread) unless its codes stream.
+inline int rt_first(int64_t M) { return M == 1 ? 1 : rt_max(M); }
 
 // Bytes between K chunks of the int8 activation buffer: 128 + 16 sigma.  The
 // K-parts that share a warp read their chunks at the same loop step; their
@@ -250,59 +251,86 @@ inline int act_stride(int Q, int P, int CPT, int threads)
     return best;
 }
 
-inline bool plan_within(int64_t N, int64_t Kc, int64_t M, int sms, int budget, Plan* out)
+// Row groups and K-parts for CTAs of R rows.
+inline bool split_rows(int64_t R, int64_t Kc, int rtmax, int64_t* RT, int64_t* Q, int64_t* P, int64_t* CPT)
 {
-    // at least 4 rows per CTA: row boundaries rounded to 4 rows then leave no CTA empty
-    const int64_t gmax = max64(1, N / 4);
-    int64_t G = min64(sms, gmax);
-    const int rtmax = rt_max(M);
-    for (int iter = 0; iter < 64; ++iter) {
-        const int64_t R = ((N + G - 1) / G + 3 + 3) & ~int64_t(3);     // rounded groups, a multiple of 4
-        if (R > (int64_t)rtmax * kMaxThreads) {
-            // rows per CTA at most ceil(N / G) + 6 after rounding
-            const int64_t cap = (int64_t)rtmax * kMaxThreads - 8;
-            G = min64(gmax, max64(G + 1, (N + cap - 1) / cap));
-            continue;
-        }
-        int64_t RT = rtmax, Q = 0, P = 0, CPT = 0;
-        for (;; RT /= 2) {
-            Q = R / RT;
-            if (Q > kMaxThreads) return false;
-            P = max64(1, min64(Kc, kMaxThreads / Q));
-            CPT = (Kc + P - 1) / P;
-            P = (Kc + CPT - 1) / CPT;
-            if (Q * P >= kMinBusyThreads || RT == 1 || R / (RT / 2) > kMaxThreads) break;
-        }
-        const int threads = kMaxThreads;
-        for (int shrink = 0; shrink < 4; ++shrink) {
-            // the bank-spreading stride when it fits, else plain 128-byte chunks
-            int S = act_stride((int)Q, (int)P, (int)CPT, (int)(Q * P));
-            int64_t smem = smem_bytes((int)M, (int)P, (int)R, Kc, S);
-            if (smem > budget && S != SHERRY_KCHUNK) {
-                S = SHERRY_KCHUNK;
-                smem = smem_bytes((int)M, (int)P, (int)R, Kc, S);
-            }
-            if (smem <= budget) {
-                if (G > 0x7fffffff) return false;
+    for (*RT = rtmax;; *RT /= 2) {
+        *Q = R / *RT;
+        if (*Q > kMaxThreads) return false;
+        *P = max64(1, min64(Kc, kMaxThreads / *Q));
+        *CPT = (Kc + *P - 1) / *P;
+        *P = (Kc + *CPT - 1) / *CPT;
+        if (*Q * *P >= kMinBusyThreads || *RT == 1 || R / (*RT / 2) > kMaxThreads) return true;
+    }
+}
+
+// The plan for G CTAs within `budget` bytes of shared memory each; false
+// when it does not fit (ring of at least two steps, or every step).
+inline bool plan_for(int64_t N, int64_t Kc, int64_t M, int64_t G, int budget, int rtmax, Plan* out)
+{
+    const int64_t R = ((N + G - 1) / G + 3 + 3) & ~int64_t(3);     // rows of a CTA at most, a multiple of 4
+    if (R > (int64_t)rtmax * kMaxThreads || G > 0x7fffffff) return false;
+    int64_t RT, Q, P, CPT;
+    if (!split_rows(R, Kc, rtmax, &RT, &Q, &P, &CPT)) return false;
+    for (int shrink = 0; shrink < 4; ++shrink) {
+        int S = act_stride((int)Q, (int)P, (int)CPT, (int)(Q * P));
+        for (int pass = 0; pass < 2; ++pass) {
+            // every step held when it fits, else the deepest ring of up to kMaxRing slots
+            int NS = (int)min64(CPT, kMaxRing);
+            const int64_t all = smem_bytes((int)M, (int)P, (int)R, (int)CPT, Kc, S);
+            if (all <= budget) NS = (int)CPT;
+            else
+                while (NS >= 2 && smem_bytes((int)M, (int)P, (int)R, NS, Kc, S) > budget) --NS;
+            if ((NS >= 2 || NS == CPT) && smem_bytes((int)M, (int)P, (int)R, NS, Kc, S) <= budget) {
                 out->G = (int)G;
                 out->R = (int)R;
                 out->RT = (int)RT;
                 out->Q = (int)Q;
                 out->P = (int)P;
                 out->CPT = (int)CPT;
-                out->threads = threads;
-                out->smem = (int)smem;
+                out->NS = NS;
+                out->threads = (int)max64(32, (Q * P + 31) / 32 * 32);
+                out->smem = smem_bytes((int)M, (int)P, (int)R, NS, Kc, S);
                 out->S = S;
                 return true;
             }
-            if (P == 1) break;
-            CPT *= 2;                                                 // fewer K-parts: fewer partial sums
-            P = (Kc + CPT - 1) / CPT;
+            if (S == SHERRY_KCHUNK) break;
+            S = SHERRY_KCHUNK;                                     // plain 128-byte activation chunks
         }
-        if (R <= 4 || G >= gmax) return false;
+        if (P == 1) break;
+        CPT *= 2;                                                  // fewer K-parts: fewer partial sums
+        P = (Kc + CPT - 1) / CPT;
+    }
+    return false;
+}
+
+inline bool plan_rt(int64_t N, int64_t Kc, int64_t M, int sms, int budget, int rtmax, Plan* out)
+{
+    // at least 4 rows per CTA: row boundaries rounded to 4 rows then leave no CTA empty
+    const int64_t gmax = max64(1, N / 4);
+    const int64_t cap = (int64_t)rtmax * kMaxThreads - 8;           // rows per CTA: at most ceil(N / G) + 6
+    int64_t G = min64(gmax, max64(sms, (N + cap - 1) / cap));
+    for (int iter = 0; iter < 64; ++iter) {
+        if (plan_for(N, Kc, M, G, budget, rtmax, out)) {
+            // codes that stream: two CTAs per SM (half the rows each) decode with twice the warps
+            Plan two;
+            if (out->NS < out->CPT && G == sms && 2 * G <= gmax && plan_for(N, Kc, M, 2 * G, budget, rtmax, &two))
+                *out = two;
+            return true;
+        }
+        if (G >= gmax) return false;
         G = min64(gmax, 2 * G);                                       // about half the rows per CTA
     }
     return false;
+}
+
+// One row per thread for one token when its codes stay resident; several rows
+// per thread otherwise (and whenever the first choice finds no plan).
+inline bool plan_within(int64_t N, int64_t Kc, int64_t M, int sms, int budget, Plan* out)
+{
+    if (rt_first(M) != rt_max(M) && plan_rt(N, Kc, M, sms, budget, rt_first(M), out) && out->NS == out->CPT)
+        return true;
+    return plan_rt(N, Kc, M, sms, budget, rt_max(M), out);
 }
 
 // The plan of a launch: within kSmemBudget (two CTAs per SM, so the next
@@ -313,74 +341,78 @@ inline bool plan(int64_t N, int64_t Kc, int64_t M, int sms, Plan* out)
     return plan_within(N, Kc, M, sms, kSmemBudget, out) || plan_within(N, Kc, M, sms, kSmemBudgetMax, out);
 }
 
+// This thread's copies of one ring step: the 16-byte pieces (4 rows of one
+// word plane) of the 4-row piece pi of part p's chunk at that step.  Row groups
+// start at multiples of 4 rows, so 4 consecutive rows of one plane are 16
+// aligned bytes in the native layout (4-byte copies for a ragged last piece).
+__device__ __forceinline__ void fetch_piece(const Params& p, int64_t r0, int Rc, int pi, int part, int step,
+                                            uint32_t slot_s)
+{
+    const int c = part * p.CPT + step;
+    if (pi < 0 || c >= (int)p.Kc) return;
+    const int64_t r = r0 + 4 * pi;
+    const int nr = min(4, Rc - 4 * pi);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(p.wnative) +
+                          ((r >> 7) * p.Kc + c) * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS);
+    const int rr = (int)(r & 127);
+    const uint32_t dst = slot_s + 4u * (uint32_t)(part * SHERRY_CHUNK_WORDS * p.R + 4 * pi);
+    if (nr == 4) {
+#pragma unroll
+        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
+            cp_async16(dst + 4u * (uint32_t)(j * p.R), src + sherry_word_pos(j, rr));
+    } else {
+        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
+            for (int e = 0; e < nr; ++e) cp_async4(dst + 4u * (uint32_t)(j * p.R + e), src + sherry_word_pos(j, rr) + e);
+    }
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Waits until at most n of this thread's committed copy groups are pending (n <= 3).
+__device__ __forceinline__ void cp_async_wait_pending(int n)
+{
+    if (n <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+    else if (n == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
+    else asm volatile("cp.async.wait_group 3;" ::: "memory");
+}
+
 template <int MT, bool FUSED, int RT>
 __global__ void __launch_bounds__(kMaxThreads, 2)
     sherry_decode_kernel(const Params p)
 {
     static_assert(RT == 1 || RT == 2 || RT == 4, "rows per thread");
+    static_assert(kMaxRing <= 4, "cp_async_wait_pending covers up to 3 pending groups");
     extern __shared__ __align__(16) uint8_t smem[];
     const int M = (int)p.M;
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int64_t r0 = row_begin(p.N, blockIdx.x, p.G), r1 = row_begin(p.N, blockIdx.x + 1, p.G);
     const int Rc = (int)(r1 - r0);
-    const int R = p.R, P = p.P, S = p.S;
+    const int R = p.R, P = p.P, S = p.S, NS = p.NS, CPT = p.CPT;
     const uint32_t s_base = ptx::smem_u32(smem);
     const uint32_t codes_s = s_base + off_codes(M, P, R);
-    const int qoff = off_q(M, P, R, p.Kc);
+    const uint32_t slot_bytes = 4u * (uint32_t)(P * SHERRY_CHUNK_WORDS * R);
+    const int qoff = off_q(M, P, R, NS);
     int8_t* qbuf = reinterpret_cast<int8_t*>(smem + qoff);
     const int QK = (int)p.Kc * S;                          // bytes per token row of qbuf
-    int32_t* sums = reinterpret_cast<int32_t*>(smem + off_sums(M, P, R));   // [M][R]
 
-    // ---- before the wait: this CTA's codes, alpha, the decode table -------------
-    // Row groups start at multiples of 4 rows, so 4 consecutive rows of one word
-    // plane are 16 aligned bytes: thread t copies 4-row piece t % R4 of every
-    // (nthr / R4)-th chunk with 16-byte cp.async (4-byte copies for a ragged end);
-    // consecutive lanes read consecutive positions of the plane.
+    // ---- before the wait: the first ring steps of this CTA's codes, alpha, the table ----
+    // Thread t copies piece pi = t % R4 of part t / R4 at every step (P * R4 <=
+    // threads: at most one piece per thread and step); consecutive lanes read
+    // consecutive positions of a plane.
+    const int R4 = (Rc + 3) >> 2;
+    const int fpi = (R4 > 0 && tid < P * R4) ? tid % R4 : -1;
+    const int fpart = R4 > 0 ? tid / R4 : 0;
+    const int first = CPT < NS ? CPT : NS;                 // steps fetched before the wait
     {
-        const int R4 = (Rc + 3) >> 2;
-        const int cstride = R4 > 0 ? nthr / R4 : 0;
-        const int pi = R4 > 0 ? tid % R4 : 0, cs = R4 > 0 ? tid / R4 : 0;
-        if (cs < cstride) {
-            const int64_t r = r0 + 4 * pi;
-            const int rr = (int)(r & 127);
-            const int nr = min(4, Rc - 4 * pi);
-            const uint32_t* src = reinterpret_cast<const uint32_t*>(p.wnative) +
-                                  (r >> 7) * p.Kc * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS);
-            int pos[SHERRY_CHUNK_WORDS];
-#pragma unroll
-            for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) pos[j] = sherry_word_pos(j, rr);
-            uint32_t dst = codes_s + 4u * (uint32_t)(cs * SHERRY_CHUNK_WORDS * R + 4 * pi);
-            const uint32_t dstep = 4u * (uint32_t)(cstride * SHERRY_CHUNK_WORDS * R);
-            for (int c = cs; c < (int)p.Kc; c += cstride) {
-                const uint32_t* sc = src + (int64_t)c * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS);
-                if (nr == 4) {
-#pragma unroll
-                    for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) cp_async16(dst + 4u * (uint32_t)(j * R), sc + pos[j]);
-                } else {
-                    for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
-                        for (int e = 0; e < nr; ++e) cp_async4(dst + 4u * (uint32_t)(j * R + e), sc + pos[j] + e);
-                }
-                dst += dstep;
-            }
-        }
         const uint32_t alpha_s = s_base + off_alpha(M, P, R);
         for (int ii = tid; ii < Rc; ii += nthr) cp_async4(alpha_s + 4u * (uint32_t)ii, p.alpha + r0 + ii);
-        asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    if constexpr (FUSED) {
-        // this CTA's share of the fp32 activations, pulled into L2 while the
-        // previous kernel finishes (a prefetch changes no value)
-        if (tid == 0) {
-            const int64_t bytes = p.M * p.K * 4;
-            const int64_t share = ((bytes + p.G - 1) / p.G + 127) & ~int64_t(127);
-            const int64_t b0 = share * blockIdx.x;
-            if (b0 < bytes)
-                bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.x) + b0,
-                                 (uint32_t)(bytes - b0 < share ? bytes - b0 : share));
-        }
+    for (int k = 0; k < first; ++k) {
+        fetch_piece(p, r0, Rc, fpi, fpart, k, codes_s + (uint32_t)k * slot_bytes);
+        cp_async_commit();
     }
-    for (int i = tid; i < M * R; i += nthr) sums[i] = 0;
     // the decode table at a 128-byte aligned shared address, so that a lookup
     // address is one LOP3: (code * 4) | table
     const uint32_t table_s = (s_base + kOffTable + 127u) & ~127u;
@@ -452,12 +484,13 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             }
         }
     } else {
+        // plain 16-byte loads, so that the copy groups in flight are the code steps only
         const int K16 = (int)(p.K >> 4);
         for (int m = 0; m < M; ++m)
-            for (int i = tid; i < K16; i += nthr)
-                cp_async16(s_base + (uint32_t)(qoff + m * QK + (i >> 3) * S + 16 * (i & 7)),
-                           p.xq + (int64_t)m * p.K + 16 * i);
-        asm volatile("cp.async.commit_group;" ::: "memory");
+            for (int i = tid; i < K16; i += nthr) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.xq + (int64_t)m * p.K) + i);
+                *reinterpret_cast<uint4*>(qbuf + m * QK + (i >> 3) * S + 16 * (i & 7)) = v;
+            }
         if (tid < M) scale_s[tid] = p.x_scale[tid];
     }
     // zero the activation tail of the last chunk: its padding codes decode to nonzero weights
@@ -469,32 +502,100 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             qbuf[m * QK + (int)(p.Kc - 1) * S + used + (i - m * tail)] = 0;
         }
     }
-    cp_async_wait_all();
+    // every step in the ring (the codes did not stream): all copies landed
+    const bool streaming = NS < CPT;
+    if (!streaming) cp_async_wait_all();
     __syncthreads();
     // the next kernel may start now: its weight prefetch overlaps this decode
     // instead of queueing in front of this CTA's activation reads
     ptx::pdl_launch_dependents();
 
-    // ---- decode + dp4a: RT rows per thread ----------------------------------------
+    // ---- decode + dp4a: RT rows per thread, one ring step at a time -----------------
+    // Step k holds chunk part * CPT + k of every part.  When the codes stream,
+    // each step waits for its own copies, a barrier makes every thread's copies
+    // visible, and after a second barrier (the slot is no longer read) the slot
+    // is refilled with step k + NS.
     const int qi = tid % p.Q, part = tid / p.Q;
     int32_t acc[RT][MT];
 #pragma unroll
     for (int r = 0; r < RT; ++r)
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[r][m] = 0;
-    if (part < P && qi * RT < Rc) {
-        const uint32_t cbase = codes_s + 4u * (uint32_t)(qi * RT);
-        const uint32_t q_s = s_base + (uint32_t)qoff;
-        const int cb = part * p.CPT;
-        const int ce = min((int)p.Kc, cb + p.CPT);
+    const bool busy = part < P && qi * RT < Rc;
+    const uint32_t q_s = s_base + (uint32_t)qoff;
+    if (RT == 1 && !streaming) {
+        // One row per thread over the whole ring (every step resident): all 32
+        // table loads of a chunk are issued before its dp4a run, and the next
+        // chunk's code words are loaded during the current one.  With the few
+        // warps a CTA has beside the next layer's prefetching CTA, this keeps
+        // more loads in flight than walking the chunk piece by piece.
+        const int nch = busy ? min(CPT, (int)p.Kc - part * CPT) : 0;
+        if (nch > 0) {
+            const uint32_t base = codes_s + 4u * (uint32_t)(part * SHERRY_CHUNK_WORDS * R + qi);
+            int32_t a4[MT][4];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) a4[m][0] = a4[m][1] = a4[m][2] = a4[m][3] = 0;
+            uint32_t wn[SHERRY_CHUNK_WORDS];
+#pragma unroll
+            for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) wn[j] = ptx::lds_u32_nv(base + 4u * (uint32_t)(j * R));
 #pragma unroll 1
-        for (int c = cb; c < ce; ++c) {
+            for (int k = 0; k < nch; ++k) {
+                uint32_t w[SHERRY_CHUNK_WORDS + 1];
+#pragma unroll
+                for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) w[j] = wn[j];
+                w[SHERRY_CHUNK_WORDS] = 0;
+                if (k + 1 < nch) {
+#pragma unroll
+                    for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
+                        wn[j] = ptx::lds_u32_nv(base + (uint32_t)(k + 1) * slot_bytes + 4u * (uint32_t)(j * R));
+                }
+                uint32_t e[32];
+#pragma unroll
+                for (int g = 0; g < 32; ++g) {
+                    const int bit = 5 * g, wi = bit >> 5, off = bit & 31;
+                    uint32_t v;
+                    if (off == 0) v = w[wi] << 2;
+                    else if (off == 1) v = w[wi] << 1;
+                    else if (off <= 27) v = w[wi] >> (off - 2);
+                    else v = __funnelshift_r(w[wi], w[wi + 1], off - 2);
+                    e[g] = ptx::lds_u32_nv((v & 0x7Cu) | table_s);
+                }
+                const uint32_t qc = q_s + (uint32_t)((part * CPT + k) * S);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    if (m >= M) break;
+#pragma unroll
+                    for (int g4 = 0; g4 < 8; ++g4) {
+                        uint32_t qv[4];
+                        lds_vec<4>(qc + (uint32_t)(m * QK + 16 * g4), qv);
+                        a4[m][0] = __dp4a((int)e[4 * g4 + 0], (int)qv[0], a4[m][0]);
+                        a4[m][1] = __dp4a((int)e[4 * g4 + 1], (int)qv[1], a4[m][1]);
+                        a4[m][2] = __dp4a((int)e[4 * g4 + 2], (int)qv[2], a4[m][2]);
+                        a4[m][3] = __dp4a((int)e[4 * g4 + 3], (int)qv[3], a4[m][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m) acc[0][m] = (a4[m][0] + a4[m][1]) + (a4[m][2] + a4[m][3]);
+        }
+    } else {
+    int committed = first;
+#pragma unroll 1
+    for (int k = 0; k < CPT; ++k) {
+        if (streaming) {
+            cp_async_wait_pending(committed - (k + 1));
+            __syncthreads();
+        }
+        const int c = part * CPT + k;
+        if (busy && c < (int)p.Kc) {
             // the five code words of each of the RT rows: one RT-word load per plane
+            const uint32_t cbase = codes_s + (uint32_t)(k % NS) * slot_bytes +
+                                   4u * (uint32_t)(part * SHERRY_CHUNK_WORDS * R + qi * RT);
             uint32_t w[RT][SHERRY_CHUNK_WORDS + 1];
 #pragma unroll
             for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) {
                 uint32_t t[RT];
-                lds_vec<RT>(cbase + 4u * (uint32_t)((c * SHERRY_CHUNK_WORDS + j) * R), t);
+                lds_vec<RT>(cbase + 4u * (uint32_t)(j * R), t);
 #pragma unroll
                 for (int r = 0; r < RT; ++r) w[r][j] = t[r];
             }
@@ -510,6 +611,14 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             piece<6, MT, RT>(w, table_s, qc, QK, M, acc);
             piece<7, MT, RT>(w, table_s, qc, QK, M, acc);
         }
+        if (streaming && k + NS < CPT) {
+            __syncthreads();
+            fetch_piece(p, r0, Rc, fpi, fpart, k + NS, codes_s + (uint32_t)(k % NS) * slot_bytes);
+            cp_async_commit();
+            ++committed;
+        }
+    }
+
     }
 
     // ---- sum the K-parts of each row, epilogue ----------------------------------------
@@ -523,23 +632,12 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
                 for (int r = 0; r < RT; ++r) red[(part * M + m) * R + qi * RT + r] = acc[r][m];
     }
     __syncthreads();
-    // output o = (token m, row i): T threads share its P parts, each adding
-    // its share into the row total with a shared atomic
     const int O = M * Rc;
-    if (O > 0) {
-        const int T = O >= nthr ? 1 : nthr / O;
-        for (int idx = tid; idx < O * T; idx += nthr) {
-            const int o = idx % O, s = idx / O;
-            const int m = o / Rc, ii = o - m * Rc;
-            int32_t v = 0;
-            for (int pp = s; pp < P; pp += T) v += red[(pp * M + m) * R + ii];
-            atomicAdd(&sums[m * R + ii], v);
-        }
-    }
-    __syncthreads();
+    // output o = (token m, row i): one thread sums its P partials
     for (int idx = tid; idx < O; idx += nthr) {
         const int m = idx / Rc, ii = idx - m * Rc;
-        const int32_t a32 = sums[m * R + ii];
+        int32_t a32 = 0;
+        for (int pp = 0; pp < P; ++pp) a32 += red[(pp * M + m) * R + ii];
         const int64_t n = r0 + ii;
         if (p.acc) p.acc[m * p.N + n] = a32;
         if (p.y) p.y[m * p.N + n] = __fmul_rn(__fmul_rn((float)a32, alpha_sm[ii]), scale_s[m]);

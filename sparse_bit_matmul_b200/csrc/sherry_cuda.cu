@@ -27,8 +27,12 @@ __device__ unsigned g_device_status = 0;
 // Activation quantiser: one CTA per token.  a = max |x| (exact), s = a / 127
 // (IEEE fp32 division), q = clamp(rint(x / s), -127, 127) with rint rounding
 // half to even; a == 0 gives s = 0 and q = 0 (the arithmetic of quant.cuh).
+// Each thread keeps its float4s in registers between the absmax and the
+// quantisation (one read of x, all loads in flight at once) when the row
+// fits (K <= 4 * kQuantXV * kQuantThreads); longer rows are read twice.
 // ---------------------------------------------------------------------------
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 512;
+constexpr int kQuantXV = 8;
 
 __global__ void __launch_bounds__(kQuantThreads)
     quant_act_kernel(const float* __restrict__ x, int64_t K, int8_t* __restrict__ q, float* __restrict__ scale)
@@ -37,29 +41,47 @@ __global__ void __launch_bounds__(kQuantThreads)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t m = blockIdx.x;
     const float4* xr = reinterpret_cast<const float4*>(x + m * K);
-    int8_t* qr = q + m * K;
-    const int64_t K4 = K / 4;
+    uint32_t* qw = reinterpret_cast<uint32_t*>(q + m * K);
+    const int K4 = (int)(K / 4);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool in_regs = K4 <= kQuantXV * kQuantThreads;
 
+    float4 v[kQuantXV];
     float a = 0.0f;
+    if (in_regs) {
+#pragma unroll
+        for (int u = 0; u < kQuantXV; ++u) {
+            const int idx = tid + u * kQuantThreads;
+            v[u] = idx < K4 ? xr[idx] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantXV; ++u) a = fmaxf(a, quant::absmax4(v[u]));
+    } else {
 #pragma unroll 4
-    for (int64_t i = threadIdx.x; i < K4; i += kQuantThreads) {
-        const float4 v = xr[i];
-        a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        for (int i = tid; i < K4; i += kQuantThreads) a = fmaxf(a, quant::absmax4(xr[i]));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     __shared__ float warp_max[kQuantThreads / 32];
-    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = a;
+    if (lane == 0) warp_max[warp] = a;
     __syncthreads();
-    a = warp_max[0];
+    // every warp combines the warp maxima: one load per lane and a shuffle tree
+    a = lane < kQuantThreads / 32 ? warp_max[lane] : 0.0f;
 #pragma unroll
-    for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, warp_max[w]);
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
 
     const quant::Scale sc = quant::make_scale(a);
-    if (threadIdx.x == 0) scale[m] = sc.s;
-    uint32_t* qw = reinterpret_cast<uint32_t*>(qr);
+    if (tid == 0) scale[m] = sc.s;
+    if (in_regs) {
+#pragma unroll
+        for (int u = 0; u < kQuantXV; ++u) {
+            const int idx = tid + u * kQuantThreads;
+            if (idx < K4) qw[idx] = quant::quantise4(v[u], sc);
+        }
+    } else {
 #pragma unroll 4
-    for (int64_t i = threadIdx.x; i < K4; i += kQuantThreads) qw[i] = quant::quantise4(xr[i], sc);
+        for (int i = tid; i < K4; i += kQuantThreads) qw[i] = quant::quantise4(xr[i], sc);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -529,6 +551,7 @@ int launch_decode(const decode::Params& p0, cudaStream_t stream)
     p.Q = pl.Q;
     p.P = pl.P;
     p.CPT = pl.CPT;
+    p.NS = pl.NS;
     p.S = pl.S;
     if (pl.smem > di.max_smem_optin) return SHERRY_ERR_DEVICE;
     if (pl.RT == 4) {

@@ -12,7 +12,8 @@
 //     of each row group, activation loads and stores, the tail, partial sums,
 //     row totals) and every native-layout word the prefetch reads stays
 //     inside its region or buffer;
-//   * every (row, K chunk) pair of a CTA is walked by exactly one thread.
+//   * every (row, K chunk) pair of a CTA is walked by exactly one thread, and
+//     every piece of every ring step is copied exactly once into its slot.
 // Prints "ok" and exits 0, or prints the first violation and exits 1.
 #include <cstdio>
 #include <cstdint>
@@ -38,21 +39,22 @@ static int check(int64_t M, int64_t N, int64_t K, int sms)
         if (M <= 8 && K <= 16384) return fail("no plan", M, N, K, sms);
         return 0;
     }
-    const int R = pl.R, RT = pl.RT, Q = pl.Q, P = pl.P, CPT = pl.CPT, S = pl.S, G = pl.G;
+    const int R = pl.R, RT = pl.RT, Q = pl.Q, P = pl.P, CPT = pl.CPT, S = pl.S, G = pl.G, NS = pl.NS;
+    if (!(NS == CPT || (NS >= 2 && NS <= decode::kMaxRing && NS < CPT))) return fail("ring slots", M, N, K, sms);
     const int nthr = pl.threads;
     if (R % 4 || R % RT || Q * RT != R || Q * P > nthr || nthr > decode::kMaxThreads || nthr % 32)
         return fail("row groups / threads", M, N, K, sms);
     if ((int64_t)P * CPT < Kc || (int64_t)(P - 1) * CPT >= Kc) return fail("K parts", M, N, K, sms);
     if (S < 128 || S % 16) return fail("activation stride", M, N, K, sms);
     const int Mi = (int)M;
-    const int o_red = decode::kOffRed, o_sums = decode::off_sums(Mi, P, R), o_alpha = decode::off_alpha(Mi, P, R);
-    const int o_codes = decode::off_codes(Mi, P, R), o_q = decode::off_q(Mi, P, R, Kc);
-    const int smem = decode::smem_bytes(Mi, P, R, Kc, S);
+    const int o_red = decode::kOffRed, o_alpha = decode::off_alpha(Mi, P, R);
+    const int o_codes = decode::off_codes(Mi, P, R), o_q = decode::off_q(Mi, P, R, NS);
+    const int smem = decode::smem_bytes(Mi, P, R, NS, Kc, S);
     if (smem != pl.smem || smem > decode::kSmemBudgetMax) return fail("smem size", M, N, K, sms);
     if (smem > decode::kSmemBudget && decode::plan_within(N, Kc, M, sms, decode::kSmemBudget, &pl))
         return fail("a two-CTA plan exists but was not taken", M, N, K, sms);
-    if (o_red + P * Mi * R * 4 > o_sums || o_sums + Mi * R * 4 > o_alpha || o_alpha + R * 4 > o_codes ||
-        o_codes + (int)Kc * 5 * R * 4 > o_q || (o_sums | o_alpha | o_codes | o_q) % 16)
+    if (o_red + P * Mi * R * 4 > o_alpha || o_alpha + R * 4 > o_codes ||
+        o_codes + NS * P * 5 * R * 4 > o_q || (o_alpha | o_codes | o_q) % 16)
         return fail("smem regions", M, N, K, sms);
     const int64_t native_words = sherry_row_tiles(N) * Kc * SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS;
     const int QK = (int)Kc * S;
@@ -63,30 +65,34 @@ static int check(int64_t M, int64_t N, int64_t K, int sms)
         const int Rc = (int)(r1 - r0);
         if (Rc < 1 || Rc > R) return fail("rows per CTA", M, N, K, sms);
         covered = r1;
-        // code prefetch: piece pi of chunk c, words j, rows 4 pi + e
+        // ring steps: thread t copies piece t % R4 of part t / R4 (t < P * R4)
+        // at every step k into slot k % NS; every (step, part, piece) exactly
+        // once, in bounds
         const int R4 = (Rc + 3) >> 2;
-        const int cstride = nthr / R4;
-        if (cstride < 1) return fail("prefetch stride", M, N, K, sms);
-        std::vector<uint8_t> got((size_t)Kc * R4, 0);
-        for (int tid = 0; tid < nthr; ++tid) {
-            const int pi = tid % R4, cs = tid / R4;
-            if (cs >= cstride) continue;
-            const int64_t r = r0 + 4 * pi;
-            const int nr = Rc - 4 * pi < 4 ? Rc - 4 * pi : 4;
-            for (int c = cs; c < (int)Kc; c += cstride) {
-                got[(size_t)c * R4 + pi]++;
+        if ((int64_t)P * R4 > nthr) return fail("more pieces than threads", M, N, K, sms);
+        std::vector<uint8_t> got((size_t)CPT * P * R4, 0);
+        for (int tid = 0; tid < P * R4; ++tid) {
+            const int fpart = tid / R4, fpi = tid % R4;
+            for (int k = 0; k < CPT; ++k) {
+                const int c = fpart * CPT + k;
+                if (c >= (int)Kc) continue;
+                got[((size_t)k * P + fpart) * R4 + fpi]++;
+                const int64_t r = r0 + 4 * fpi;
+                const int nr = Rc - 4 * fpi < 4 ? Rc - 4 * fpi : 4;
+                if (((r & 127) + nr - 1) > 127) return fail("piece crosses a tile", M, N, K, sms);
                 for (int j = 0; j < 5; ++j) {
-                    const int64_t src = (r >> 7) * Kc * 640 + (int64_t)c * 640 + sherry_word_pos(j, (int)(r & 127));
+                    const int64_t src = ((r >> 7) * Kc + c) * 640 + sherry_word_pos(j, (int)(r & 127));
                     if (src < 0 || src + nr > native_words) return fail("prefetch source", M, N, K, sms);
-                    // rows of a piece are consecutive words of the plane unless the piece crosses a tile
-                    if (((r & 127) + nr - 1) > 127) return fail("piece crosses a tile", M, N, K, sms);
-                    const int64_t dst = (int64_t)(c * 5 + j) * R + 4 * pi;
-                    if (dst < 0 || dst + nr > Kc * 5 * R) return fail("prefetch destination", M, N, K, sms);
+                    const int64_t dst = (int64_t)(k % NS) * P * 5 * R + (int64_t)(fpart * 5 + j) * R + 4 * fpi;
+                    if (dst < 0 || dst + nr > (int64_t)NS * P * 5 * R) return fail("prefetch destination", M, N, K, sms);
                 }
             }
         }
-        for (uint8_t g : got)
-            if (g != 1) return fail("prefetch pieces not copied exactly once", M, N, K, sms);
+        for (int k = 0; k < CPT; ++k)
+            for (int pp = 0; pp < P; ++pp)
+                for (int pi = 0; pi < R4; ++pi)
+                    if (got[((size_t)k * P + pp) * R4 + pi] != (pp * CPT + k < (int)Kc ? 1 : 0))
+                        return fail("step pieces not copied exactly once", M, N, K, sms);
         // main loop and partial sums
         std::vector<uint8_t> walk((size_t)Rc * Kc, 0);
         for (int tid = 0; tid < nthr; ++tid) {
@@ -97,12 +103,13 @@ static int check(int64_t M, int64_t N, int64_t K, int sms)
                 if (red >= (int64_t)P * Mi * R) return fail("partial sums index", M, N, K, sms);
             }
             if (qi * RT >= Rc) continue;
-            const int cb = part * CPT, ce = cb + CPT < (int)Kc ? cb + CPT : (int)Kc;
-            if (cb >= ce) return fail("empty K part", M, N, K, sms);
-            for (int c = cb; c < ce; ++c) {
+            if (part * CPT >= (int)Kc) return fail("empty K part", M, N, K, sms);
+            for (int k = 0; k < CPT; ++k) {
+                const int c = part * CPT + k;
+                if (c >= (int)Kc) continue;
                 for (int j = 0; j < 5; ++j) {
-                    const int64_t w = (int64_t)(c * 5 + j) * R + qi * RT;
-                    if (w + RT > Kc * 5 * R) return fail("code load", M, N, K, sms);
+                    const int64_t w = (int64_t)(k % NS) * P * 5 * R + (int64_t)(part * 5 + j) * R + qi * RT;
+                    if (w + RT > (int64_t)NS * P * 5 * R) return fail("code load", M, N, K, sms);
                 }
                 const int64_t a = (int64_t)(Mi - 1) * QK + (int64_t)c * S + 16 * 7 + 16;
                 if (a > (int64_t)Mi * QK) return fail("activation load", M, N, K, sms);
