@@ -118,6 +118,10 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -141,6 +145,26 @@ template <>
 __device__ __forceinline__ void lds_vec<4>(uint32_t addr, uint32_t (&v)[4])
 {
     asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]) : "r"(addr));
+}
+
+// The same loads, kept in program order with this thread's copies into the
+// ring (volatile: a refill of the slot is never issued ahead of them).
+template <int N>
+__device__ __forceinline__ void lds_vec_ordered(uint32_t addr, uint32_t (&v)[N]);
+template <>
+__device__ __forceinline__ void lds_vec_ordered<1>(uint32_t addr, uint32_t (&v)[1])
+{
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v[0]) : "r"(addr));
+}
+template <>
+__device__ __forceinline__ void lds_vec_ordered<2>(uint32_t addr, uint32_t (&v)[2])
+{
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v[0]), "=r"(v[1]) : "r"(addr));
+}
+template <>
+__device__ __forceinline__ void lds_vec_ordered<4>(uint32_t addr, uint32_t (&v)[4])
+{
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]) : "r"(addr));
 }
 
 // Byte offset, in the table, of group g's code within a row's five chunk
@@ -366,6 +390,37 @@ __device__ __forceinline__ void fetch_piece(const Params& p, int64_t r0, int Rc,
     }
 }
 
+// Streaming rings: the code words a thread decodes at one step (rows row0 ..
+// row0 + RT - 1 of the CTA, part `part`'s chunk at that step, five planes),
+// copied by that thread itself, so that waiting for its own copy groups is
+// all the synchronisation the ring needs.  row0 is a multiple of RT and the
+// CTA's first row a multiple of 4, so the RT words of a plane are 4 RT
+// aligned bytes in the native layout (4-byte copies for a ragged last group).
+template <int RT>
+__device__ __forceinline__ void fetch_own(const Params& p, int64_t r0, int Rc, int row0, int part, int step,
+                                          uint32_t slot_s)
+{
+    const int c = part * p.CPT + step;
+    if (row0 >= Rc || c >= (int)p.Kc) return;
+    const int64_t r = r0 + row0;
+    const int nr = min(RT, Rc - row0);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(p.wnative) +
+                          ((r >> 7) * p.Kc + c) * (SHERRY_CHUNK_WORDS * SHERRY_TILE_ROWS);
+    const int rr = (int)(r & 127);
+    const uint32_t dst = slot_s + 4u * (uint32_t)(part * SHERRY_CHUNK_WORDS * p.R + row0);
+    if (nr == RT) {
+#pragma unroll
+        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) {
+            if constexpr (RT == 4) cp_async16(dst + 4u * (uint32_t)(j * p.R), src + sherry_word_pos(j, rr));
+            else if constexpr (RT == 2) cp_async8(dst + 4u * (uint32_t)(j * p.R), src + sherry_word_pos(j, rr));
+            else cp_async4(dst + 4u * (uint32_t)(j * p.R), src + sherry_word_pos(j, rr));
+        }
+    } else {
+        for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j)
+            for (int e = 0; e < nr; ++e) cp_async4(dst + 4u * (uint32_t)(j * p.R + e), src + sherry_word_pos(j, rr) + e);
+    }
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 // Waits until at most n of this thread's committed copy groups are pending (n <= 3).
@@ -398,9 +453,19 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     const int QK = (int)p.Kc * S;                          // bytes per token row of qbuf
 
     // ---- before the wait: the first ring steps of this CTA's codes, alpha, the table ----
-    // Thread t copies piece pi = t % R4 of part t / R4 at every step (P * R4 <=
-    // threads: at most one piece per thread and step); consecutive lanes read
-    // consecutive positions of a plane.
+    // Thread (qi, part) decodes rows qi * RT .. qi * RT + RT - 1 of K part `part`.
+    // Resident rings (every step fits): thread t copies piece pi = t % R4 of
+    // part t / R4 at every step (P * R4 <= threads: at most one piece per
+    // thread and step), consecutive lanes reading consecutive positions of a
+    // plane, and one barrier publishes them.  Streaming rings of 4 rows per
+    // thread: every thread copies what it decodes (fetch_own, one 16-byte copy
+    // per plane), so steps need no barrier; with 1 or 2 rows per thread the
+    // pieces are copied as for resident rings and two barriers a step publish
+    // and release them (smaller own copies measured slower there).
+    const bool streaming = NS < CPT;
+    const bool own = streaming && RT == 4;
+    const int qi = tid % p.Q, part = tid / p.Q;
+    const bool busy = part < P && qi * RT < Rc;
     const int R4 = (Rc + 3) >> 2;
     const int fpi = (R4 > 0 && tid < P * R4) ? tid % R4 : -1;
     const int fpart = R4 > 0 ? tid / R4 : 0;
@@ -410,7 +475,8 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
         for (int ii = tid; ii < Rc; ii += nthr) cp_async4(alpha_s + 4u * (uint32_t)ii, p.alpha + r0 + ii);
     }
     for (int k = 0; k < first; ++k) {
-        fetch_piece(p, r0, Rc, fpi, fpart, k, codes_s + (uint32_t)k * slot_bytes);
+        if (!own) fetch_piece(p, r0, Rc, fpi, fpart, k, codes_s + (uint32_t)k * slot_bytes);
+        else if (busy) fetch_own<RT>(p, r0, Rc, qi * RT, part, k, codes_s + (uint32_t)k * slot_bytes);
         cp_async_commit();
     }
     // the decode table at a 128-byte aligned shared address, so that a lookup
@@ -503,7 +569,6 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
         }
     }
     // every step in the ring (the codes did not stream): all copies landed
-    const bool streaming = NS < CPT;
     if (!streaming) cp_async_wait_all();
     __syncthreads();
     // the next kernel may start now: its weight prefetch overlaps this decode
@@ -512,16 +577,15 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
 
     // ---- decode + dp4a: RT rows per thread, one ring step at a time -----------------
     // Step k holds chunk part * CPT + k of every part.  When the codes stream,
-    // each step waits for its own copies, a barrier makes every thread's copies
-    // visible, and after a second barrier (the slot is no longer read) the slot
-    // is refilled with step k + NS.
-    const int qi = tid % p.Q, part = tid / p.Q;
+    // each thread waits for its own copies of step k; with own copies it
+    // decodes the step and refills the slot with its rows of step k + NS,
+    // otherwise a barrier makes every thread's copies visible first and a
+    // second one (the slot is no longer read) precedes the refill.
     int32_t acc[RT][MT];
 #pragma unroll
     for (int r = 0; r < RT; ++r)
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[r][m] = 0;
-    const bool busy = part < P && qi * RT < Rc;
     const uint32_t q_s = s_base + (uint32_t)qoff;
     if (RT == 1 && !streaming) {
         // One row per thread over the whole ring (every step resident): all 32
@@ -584,7 +648,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     for (int k = 0; k < CPT; ++k) {
         if (streaming) {
             cp_async_wait_pending(committed - (k + 1));
-            __syncthreads();
+            if (!own) __syncthreads();
         }
         const int c = part * CPT + k;
         if (busy && c < (int)p.Kc) {
@@ -595,7 +659,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
 #pragma unroll
             for (int j = 0; j < SHERRY_CHUNK_WORDS; ++j) {
                 uint32_t t[RT];
-                lds_vec<RT>(cbase + 4u * (uint32_t)(j * R), t);
+                lds_vec_ordered<RT>(cbase + 4u * (uint32_t)(j * R), t);
 #pragma unroll
                 for (int r = 0; r < RT; ++r) w[r][j] = t[r];
             }
@@ -612,8 +676,12 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             piece<7, MT, RT>(w, table_s, qc, QK, M, acc);
         }
         if (streaming && k + NS < CPT) {
-            __syncthreads();
-            fetch_piece(p, r0, Rc, fpi, fpart, k + NS, codes_s + (uint32_t)(k % NS) * slot_bytes);
+            if (own) {
+                if (busy) fetch_own<RT>(p, r0, Rc, qi * RT, part, k + NS, codes_s + (uint32_t)(k % NS) * slot_bytes);
+            } else {
+                __syncthreads();
+                fetch_piece(p, r0, Rc, fpi, fpart, k + NS, codes_s + (uint32_t)(k % NS) * slot_bytes);
+            }
             cp_async_commit();
             ++committed;
         }

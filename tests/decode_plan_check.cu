@@ -65,34 +65,68 @@ static int check(int64_t M, int64_t N, int64_t K, int sms)
         const int Rc = (int)(r1 - r0);
         if (Rc < 1 || Rc > R) return fail("rows per CTA", M, N, K, sms);
         covered = r1;
-        // ring steps: thread t copies piece t % R4 of part t / R4 (t < P * R4)
-        // at every step k into slot k % NS; every (step, part, piece) exactly
-        // once, in bounds
-        const int R4 = (Rc + 3) >> 2;
-        if ((int64_t)P * R4 > nthr) return fail("more pieces than threads", M, N, K, sms);
-        std::vector<uint8_t> got((size_t)CPT * P * R4, 0);
-        for (int tid = 0; tid < P * R4; ++tid) {
-            const int fpart = tid / R4, fpi = tid % R4;
-            for (int k = 0; k < CPT; ++k) {
-                const int c = fpart * CPT + k;
-                if (c >= (int)Kc) continue;
-                got[((size_t)k * P + fpart) * R4 + fpi]++;
-                const int64_t r = r0 + 4 * fpi;
-                const int nr = Rc - 4 * fpi < 4 ? Rc - 4 * fpi : 4;
-                if (((r & 127) + nr - 1) > 127) return fail("piece crosses a tile", M, N, K, sms);
-                for (int j = 0; j < 5; ++j) {
-                    const int64_t src = ((r >> 7) * Kc + c) * 640 + sherry_word_pos(j, (int)(r & 127));
-                    if (src < 0 || src + nr > native_words) return fail("prefetch source", M, N, K, sms);
-                    const int64_t dst = (int64_t)(k % NS) * P * 5 * R + (int64_t)(fpart * 5 + j) * R + 4 * fpi;
-                    if (dst < 0 || dst + nr > (int64_t)NS * P * 5 * R) return fail("prefetch destination", M, N, K, sms);
+        if (NS == CPT || RT != 4) {
+            // ring steps: thread t copies piece t % R4 of part t / R4 (t < P * R4)
+            // at every step k into slot k % NS; every (step, part, piece) exactly
+            // once, in bounds
+            const int R4 = (Rc + 3) >> 2;
+            if ((int64_t)P * R4 > nthr) return fail("more pieces than threads", M, N, K, sms);
+            std::vector<uint8_t> got((size_t)CPT * P * R4, 0);
+            for (int tid = 0; tid < P * R4; ++tid) {
+                const int fpart = tid / R4, fpi = tid % R4;
+                for (int k = 0; k < CPT; ++k) {
+                    const int c = fpart * CPT + k;
+                    if (c >= (int)Kc) continue;
+                    got[((size_t)k * P + fpart) * R4 + fpi]++;
+                    const int64_t r = r0 + 4 * fpi;
+                    const int nr = Rc - 4 * fpi < 4 ? Rc - 4 * fpi : 4;
+                    if (((r & 127) + nr - 1) > 127) return fail("piece crosses a tile", M, N, K, sms);
+                    for (int j = 0; j < 5; ++j) {
+                        const int64_t src = ((r >> 7) * Kc + c) * 640 + sherry_word_pos(j, (int)(r & 127));
+                        if (src < 0 || src + nr > native_words) return fail("prefetch source", M, N, K, sms);
+                        const int64_t dst = (int64_t)(k % NS) * P * 5 * R + (int64_t)(fpart * 5 + j) * R + 4 * fpi;
+                        if (dst < 0 || dst + nr > (int64_t)NS * P * 5 * R) return fail("prefetch destination", M, N, K, sms);
+                    }
                 }
             }
+            for (int k = 0; k < CPT; ++k)
+                for (int pp = 0; pp < P; ++pp)
+                    for (int pi = 0; pi < R4; ++pi)
+                        if (got[((size_t)k * P + pp) * R4 + pi] != (pp * CPT + k < (int)Kc ? 1 : 0))
+                            return fail("step pieces not copied exactly once", M, N, K, sms);
+        } else {
+            // streaming ring of 4 rows per thread: thread (qi, part) copies its
+            // own rows of every step (row0 = qi * RT, ragged last group in 4-byte words); every
+            // (step, part, row) exactly once, in bounds, RT-word aligned
+            std::vector<uint8_t> got((size_t)CPT * P * Rc, 0);
+            for (int tid = 0; tid < nthr; ++tid) {
+                const int qi = tid % Q, part = tid / Q;
+                if (part >= P || qi * RT >= Rc) continue;
+                const int row0 = qi * RT, nr = Rc - row0 < RT ? Rc - row0 : RT;
+                const int64_t r = r0 + row0;
+                if (((r & 127) + nr - 1) > 127) return fail("own rows cross a tile", M, N, K, sms);
+                for (int k = 0; k < CPT; ++k) {
+                    const int c = part * CPT + k;
+                    if (c >= (int)Kc) continue;
+                    for (int e = 0; e < nr; ++e) got[((size_t)k * P + part) * Rc + row0 + e]++;
+                    for (int j = 0; j < 5; ++j) {
+                        const int64_t src = ((r >> 7) * Kc + c) * 640 + sherry_word_pos(j, (int)(r & 127));
+                        if (src < 0 || src + nr > native_words) return fail("own copy source", M, N, K, sms);
+                        const int64_t dst = (int64_t)(k % NS) * P * 5 * R + (int64_t)(part * 5 + j) * R + row0;
+                        if (dst < 0 || dst + nr > (int64_t)NS * P * 5 * R) return fail("own copy destination", M, N, K, sms);
+                        if (nr == RT && (src % RT || dst % RT)) return fail("own copy alignment", M, N, K, sms);
+                        for (int e = 1; e < nr; ++e)
+                            if (((r >> 7) * Kc + c) * 640 + sherry_word_pos(j, (int)((r + e) & 127)) != src + e)
+                                return fail("own rows not consecutive", M, N, K, sms);
+                    }
+                }
+            }
+            for (int k = 0; k < CPT; ++k)
+                for (int pp = 0; pp < P; ++pp)
+                    for (int rr = 0; rr < Rc; ++rr)
+                        if (got[((size_t)k * P + pp) * Rc + rr] != (pp * CPT + k < (int)Kc ? 1 : 0))
+                            return fail("step rows not copied exactly once", M, N, K, sms);
         }
-        for (int k = 0; k < CPT; ++k)
-            for (int pp = 0; pp < P; ++pp)
-                for (int pi = 0; pi < R4; ++pi)
-                    if (got[((size_t)k * P + pp) * R4 + pi] != (pp * CPT + k < (int)Kc ? 1 : 0))
-                        return fail("step pieces not copied exactly once", M, N, K, sms);
         // main loop and partial sums
         std::vector<uint8_t> walk((size_t)Rc * Kc, 0);
         for (int tid = 0; tid < nthr; ++tid) {
