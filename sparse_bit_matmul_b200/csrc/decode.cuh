@@ -432,6 +432,76 @@ __device__ __forceinline__ void cp_async_wait_pending(int n)
     else asm volatile("cp.async.wait_group 3;" ::: "memory");
 }
 
+// The fused activation phase: per token, absmax over the row, s = a / 127 and
+// int8 codes into the shared activation buffer (qbuf: token m's K chunk c at
+// byte m * QK + c * S), scales into scale_s.  XV float4 slots per thread hold
+// the row in registers (all loads in flight at once); XV = 0 streams it from
+// global memory twice.  Whether the row is in registers is a compile-time
+// property of each instantiation.
+template <int XV>
+__device__ __forceinline__ void fused_activations(const Params& p, int8_t* qbuf, int QK, int S, float* scale_s,
+                                                  float* warp_max, int M, int K4)
+{
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const int nwarps = (nthr + 31) >> 5;
+    constexpr bool in_regs = XV > 0;
+    constexpr int NV = XV > 0 ? XV : 1;
+    for (int m = 0; m < M; ++m) {
+        const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)m * p.K);
+        int8_t* qr = qbuf + m * QK;
+        float4 v[NV];
+        float mx = 0.0f;
+        if constexpr (in_regs) {
+            // predicated loads, all in flight at once; slots past the row
+            // hold zeros, which leave the maximum unchanged
+#pragma unroll
+            for (int u = 0; u < XV; ++u) {
+                const int idx = tid + u * nthr;
+                v[u] = idx < K4 ? xr[idx] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+#pragma unroll
+            for (int u = 0; u < XV; ++u) mx = fmaxf(mx, quant::absmax4(v[u]));
+        } else {
+#pragma unroll 4
+            for (int i = tid; i < K4; i += nthr) mx = fmaxf(mx, quant::absmax4(xr[i]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) warp_max[(m & 1) * 16 + warp] = mx;
+        __syncthreads();
+        // every warp combines the (at most 16) warp maxima: one load per
+        // lane and a shuffle tree, not a chain of dependent loads
+        float a = lane < nwarps ? warp_max[(m & 1) * 16 + lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        const quant::Scale sc = quant::make_scale(a);
+        if (tid == 0) {
+            scale_s[m] = sc.s;
+            if (p.xs_out && blockIdx.x == 0) p.xs_out[m] = sc.s;
+        }
+        uint32_t* qo = (p.xq_out && blockIdx.x == 0) ? reinterpret_cast<uint32_t*>(p.xq_out + (int64_t)m * p.K)
+                                                      : nullptr;
+        // word idx (activations 4 idx .. 4 idx + 3) sits in chunk idx / 32
+        if constexpr (in_regs) {
+#pragma unroll
+            for (int u = 0; u < XV; ++u) {
+                const int idx = tid + u * nthr;
+                if (idx < K4) {
+                    const uint32_t w = quant::quantise4(v[u], sc);
+                    *reinterpret_cast<uint32_t*>(qr + (idx >> 5) * S + 4 * (idx & 31)) = w;
+                    if (qo) qo[idx] = w;
+                }
+            }
+        } else {
+            for (int i = tid; i < K4; i += nthr) {
+                const uint32_t w = quant::quantise4(xr[i], sc);
+                *reinterpret_cast<uint32_t*>(qr + (i >> 5) * S + 4 * (i & 31)) = w;
+                if (qo) qo[i] = w;
+            }
+        }
+    }
+}
+
 template <int MT, bool FUSED, int RT>
 __global__ void __launch_bounds__(kMaxThreads, 2)
     sherry_decode_kernel(const Params p)
@@ -490,65 +560,11 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     float* scale_s = reinterpret_cast<float*>(smem + kOffScale);
     const int K4 = (int)(p.K >> 2);
     if constexpr (FUSED) {
-        // per token: the thread's float4s stay in registers (all loads in
-        // flight at once), block absmax, then quantise from the registers
+        // rows of up to kXV float4s per thread are held in registers; longer
+        // rows stream from global memory (XV = 0)
         float* warp_max = reinterpret_cast<float*>(smem + kOffWarpMax);
-        const int nwarps = (nthr + 31) >> 5;
-        const bool in_regs = K4 <= kXV * nthr;
-        for (int m = 0; m < M; ++m) {
-            const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)m * p.K);
-            int8_t* qr = qbuf + m * QK;
-            float4 v[kXV];
-            float mx = 0.0f;
-            if (in_regs) {
-                // predicated loads, all in flight at once; slots past the row
-                // hold zeros, which leave the maximum unchanged
-#pragma unroll
-                for (int u = 0; u < kXV; ++u) {
-                    const int idx = tid + u * nthr;
-                    v[u] = idx < K4 ? xr[idx] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                }
-#pragma unroll
-                for (int u = 0; u < kXV; ++u) mx = fmaxf(mx, quant::absmax4(v[u]));
-            } else {
-#pragma unroll 4
-                for (int i = tid; i < K4; i += nthr) mx = fmaxf(mx, quant::absmax4(xr[i]));
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0) warp_max[(m & 1) * 16 + warp] = mx;
-            __syncthreads();
-            // every warp combines the (at most 16) warp maxima: one load per
-            // lane and a shuffle tree, not a chain of dependent loads
-            float a = lane < nwarps ? warp_max[(m & 1) * 16 + lane] : 0.0f;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            const quant::Scale sc = quant::make_scale(a);
-            if (tid == 0) {
-                scale_s[m] = sc.s;
-                if (p.xs_out && blockIdx.x == 0) p.xs_out[m] = sc.s;
-            }
-            uint32_t* qo = (p.xq_out && blockIdx.x == 0) ? reinterpret_cast<uint32_t*>(p.xq_out + (int64_t)m * p.K)
-                                                          : nullptr;
-            // word idx (activations 4 idx .. 4 idx + 3) sits in chunk idx / 32
-            if (in_regs) {
-#pragma unroll
-                for (int u = 0; u < kXV; ++u) {
-                    const int idx = tid + u * nthr;
-                    if (idx < K4) {
-                        const uint32_t w = quant::quantise4(v[u], sc);
-                        *reinterpret_cast<uint32_t*>(qr + (idx >> 5) * S + 4 * (idx & 31)) = w;
-                        if (qo) qo[idx] = w;
-                    }
-                }
-            } else {
-                for (int i = tid; i < K4; i += nthr) {
-                    const uint32_t w = quant::quantise4(xr[i], sc);
-                    *reinterpret_cast<uint32_t*>(qr + (i >> 5) * S + 4 * (i & 31)) = w;
-                    if (qo) qo[i] = w;
-                }
-            }
-        }
+        if (K4 <= kXV * nthr) fused_activations<kXV>(p, qbuf, QK, S, scale_s, warp_max, M, K4);
+        else fused_activations<0>(p, qbuf, QK, S, scale_s, warp_max, M, K4);
     } else {
         // plain 16-byte loads, so that the copy groups in flight are the code steps only
         const int K16 = (int)(p.K >> 4);
