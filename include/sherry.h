@@ -183,7 +183,13 @@ int sherry_gemm_acc(const int8_t* x_i8, const float* x_scale, const void* Wnativ
  * into tensor memory (one 32-bit cell per group of 4) and multiplied with
  * tcgen05.mma kind::i8 against the int8 activations (TMA-loaded, 128-byte
  * swizzle); K is split over all SMs with exact int32 partial sums in the
- * per-device workspace.  Arguments as sherry_gemm_acc.
+ * per-device workspace.  Launched with programmatic dependent launch: the
+ * codes of each CTA's first pipeline round are copied before the previous
+ * kernel on the stream ends; activations, scales and outputs are touched
+ * only after it completed.  So, as for sherry_gemm_decode, Wnative must not
+ * be written by the kernel launched just before on the same stream unless
+ * that kernel ends without triggering its dependents early (every ordinary
+ * kernel, and sherry_repack, does so).  Arguments as sherry_gemm_acc.
  */
 int sherry_gemm_tc(const int8_t* x_i8, const float* x_scale, const void* Wnative,
                    const float* alpha, float* y, int32_t* acc, int64_t M, int64_t N,

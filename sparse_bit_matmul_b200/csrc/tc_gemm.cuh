@@ -342,6 +342,33 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
         // Converged warp, elected-lane issue and a non-blocking test of the
         // next slot, for the same reason as the MMA loop below: a copy issued
         // late delays every role after it.
+        //
+        // The codes do not depend on the previous kernel: the first ring
+        // round's code copies (each with its stage's whole byte count) are
+        // issued before the dependency wait, so that they overlap the end of
+        // the previous kernel; their activation boxes follow after the wait.
+        int64_t npre = 0;
+        {
+            SegWalk w(p, blockIdx.x, G);
+            while (!w.done() && npre < C::kStages) {
+                const int64_t tn = w.tile % p.TN;
+                int c = (int)w.cb;
+                int left = (int)(w.ce - w.cb);
+                while (left > 0 && npre < C::kStages) {
+                    const int nch = left < SC ? left : SC;
+                    const uint32_t st = (uint32_t)npre;          // first round: slot npre, no wait
+                    ptx::mbar_arrive_expect_tx_elect(full_bar((int)st),
+                                                     (uint32_t)(nch * (C::kChunkWBytes + C::kBChunkBytes)));
+                    ptx::bulk_g2s_elect(sbase + C::kOffCodes + st * C::kCodeStageBytes,
+                                        p.wnative + (tn * p.Kc + c) * (int64_t)C::kChunkWBytes,
+                                        (uint32_t)(nch * C::kChunkWBytes), full_bar((int)st));
+                    c += nch;
+                    left -= nch;
+                    ++npre;
+                }
+                w.next();
+            }
+        }
         ptx::pdl_wait();
         int s = 0;
         uint32_t ph = 0;
@@ -357,16 +384,20 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
             int left = (int)(w.ce - w.cb);
             while (left > 0) {
                 const int nch = left < SC ? left : SC;
-                if (!ready) {
+                const bool pre = issued < npre;      // codes already in flight, empty(s) fresh
+                if (!ready && !pre) {
                     ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs));
                     if (!ok) break;
                 }
                 const int s1 = (s + 1 == C::kStages) ? 0 : s + 1;
                 const uint32_t ph1 = (s + 1 == C::kStages) ? ph ^ 1u : ph;
                 const uint32_t t_e = ptx::mbar_test(empty_bar(s1), ph1 ^ 1u);
-                ptx::mbar_arrive_expect_tx_elect(full_bar(s), (uint32_t)(nch * (C::kChunkWBytes + C::kBChunkBytes)));
-                ptx::bulk_g2s_elect(sbase + C::kOffCodes + (uint32_t)s * C::kCodeStageBytes, src,
-                                    (uint32_t)(nch * C::kChunkWBytes), full_bar(s));
+                if (!pre) {
+                    ptx::mbar_arrive_expect_tx_elect(full_bar(s),
+                                                     (uint32_t)(nch * (C::kChunkWBytes + C::kBChunkBytes)));
+                    ptx::bulk_g2s_elect(sbase + C::kOffCodes + (uint32_t)s * C::kCodeStageBytes, src,
+                                        (uint32_t)(nch * C::kChunkWBytes), full_bar(s));
+                }
                 if (nch == SC) {
 #pragma unroll
                     for (int j = 0; j < SC; ++j)
