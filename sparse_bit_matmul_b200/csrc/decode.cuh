@@ -53,7 +53,7 @@ constexpr int kMaxM = 8;
 constexpr int kMaxThreads = 512;
 constexpr int kSmemBudget = 100 * 1024;     // two CTAs (this layer, the next) per SM
 constexpr int kSmemBudgetMax = 200 * 1024;  // one CTA per SM: shapes whose activations alone need more
-constexpr int kXV = 8;                      // fused: float4 activations per thread held in registers
+constexpr int kXV = 7;                      // fused: float4 activations per thread held in registers (K <= 14336 at 512 threads)
 
 struct Params {
     const uint8_t* wnative;

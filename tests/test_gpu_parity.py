@@ -124,7 +124,10 @@ SMALL = [(1, 128, 256), (1, 37, 96), (3, 300, 4096), (17, 129, 224), (33, 200, 5
          # shares over many CTAs (128- and 64-token tiles)
          (130, 384, 14336), (40, 256, 14336),
          # 192-token tiles (M >= 1536), the last one ragged
-         (1600, 300, 512)]
+         (1600, 300, 512),
+         # one token with rows longer than the fused quantiser holds in
+         # registers (K / 4 > 7 float4s per thread): x streams from memory
+         (1, 300, 16384), (1, 4100, 16384)]
 
 
 def _kernel_serves(kernel: str, M: int, K: int) -> bool:
