@@ -371,6 +371,58 @@ def time_graph(g, steps: int, warmup: int, world: int, sampler=None):
     return e0.elapsed_time(e1) / 1e3
 
 
+def time_pipelined_e2e(g_comp, x_dev, x_host, y_dev, y_host, steps: int, warmup: int, world: int):
+    """End-to-end steps with the copies overlapped, as a serving loop runs them:
+    step k's inputs go host -> device on one copy stream while step k - 1
+    computes, its outputs device -> host on another while step k + 1 computes.
+    Two device buffers of inputs and of outputs (b = k mod 2); g_comp[b] is the
+    captured compute of one step on buffer pair b.  Every step still copies
+    its own inputs in and its own outputs out inside the timed region, which
+    runs from before the first input copy to after the last output copy."""
+    import torch
+    comp = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event(), torch.cuda.Event()]
+    ev_comp = [torch.cuda.Event(), torch.cuda.Event()]
+    ev_out = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def run(n):
+        used = [False, False]
+        for k in range(n):
+            b = k & 1
+            if used[b]:
+                h2d.wait_event(ev_comp[b])            # step k - 2 has read x_dev[b]
+            with torch.cuda.stream(h2d):
+                x_dev[b].copy_(x_host, non_blocking=True)
+            ev_in[b].record(h2d)
+            comp.wait_event(ev_in[b])
+            if used[b]:
+                comp.wait_event(ev_out[b])            # step k - 2's outputs have left y_dev[b]
+            g_comp[b].replay()
+            ev_comp[b].record(comp)
+            d2h.wait_event(ev_comp[b])
+            with torch.cuda.stream(d2h):
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+            ev_out[b].record(d2h)
+            used[b] = True
+        for b in range(min(n, 2)):
+            comp.wait_event(ev_out[b])
+
+    run(max(warmup, 2))
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    h2d.wait_event(e0)
+    d2h.wait_event(e0)
+    run(steps)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1) / 1e3
+
+
 def run_gpu(args, world, rank, local):
     import torch
     import sparse_bit_matmul_b200 as sbm
@@ -439,6 +491,26 @@ def run_gpu(args, world, rank, local):
             layer(L, L["x_step"], L["y_step"])
         Y_host.copy_(Y_dev, non_blocking=True)
 
+    # the pipelined end-to-end form: two device buffer pairs, the compute of
+    # one step on each captured as its own graph
+    X_dev2 = [X_dev, torch.empty_like(X_dev)]
+    Y_dev2 = [Y_dev, torch.empty_like(Y_dev)]
+    Y_host2 = [Y_host, torch.empty(y_total, dtype=torch.float32).pin_memory()]
+    pipe_views = []
+    for b in range(2):
+        xo = yo = 0
+        vb = []
+        for L in layers:
+            nx, ny = L["x"].numel(), L["y"].numel()
+            vb.append((X_dev2[b][xo:xo + nx].view(L["x"].shape), Y_dev2[b][yo:yo + ny].view(L["y"].shape)))
+            xo += nx
+            yo += ny
+        pipe_views.append(vb)
+
+    def compute_on(b):
+        for L, (xv, yv) in zip(layers, pipe_views[b]):
+            layer(L, xv, yv)
+
     def e2e_per_layer_step():
         for L in layers:
             L["x"].copy_(L["x_host"], non_blocking=True)
@@ -453,6 +525,7 @@ def run_gpu(args, world, rank, local):
     g_two = capture(two_launch_step) if fused else None
     g_e2e = capture(e2e_step)
     g_e2e_layer = capture(e2e_per_layer_step)
+    g_comp = [capture(lambda: compute_on(0)), capture(lambda: compute_on(1))]
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -464,6 +537,8 @@ def run_gpu(args, world, rank, local):
     t_two = max_over_ranks(time_graph(g_two, args.steps, args.warmup, world), world) if fused else None
     t_e2e = max_over_ranks(time_graph(g_e2e, args.steps, args.warmup, world), world)
     t_e2e_layer = max_over_ranks(time_graph(g_e2e_layer, args.steps, args.warmup, world), world)
+    t_e2e_pipe = max_over_ranks(time_pipelined_e2e(g_comp, X_dev2, X_host, Y_dev2, Y_host2, args.steps,
+                                                   args.warmup, world), world)
     assert sbm.last_device_status() == 0, "a kernel reported a bounded wait running out"
 
     peaks, peak_src = load_peaks()
@@ -511,18 +586,24 @@ def run_gpu(args, world, rank, local):
             "gemm_gbs": round(step_bytes / (t_gemm / args.steps) / 1e9, 2),
             "two_launch_step_gbs": (round(step_bytes * args.steps / t_two / 1e9, 2) if fused else None),
         },
-        "e2e": {"value": round(step_bytes * world * args.steps / t_e2e / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(step_bytes * world * args.steps / t_e2e_pipe / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "path": ("one pinned host buffer of the step's layer inputs -> one H2D copy -> "
+                "path": ("per step: one H2D copy of the step's layer inputs from one pinned host buffer "
+                         "(copy stream 1) -> "
                          + ("sherry_linear" if fused else f"sherry_quant_act -> sherry_gemm[{kernel}]")
-                         + " per layer on device views -> one D2H copy of the step's outputs, "
-                         "in one CUDA graph per step"),
+                         + " per layer on device views (one CUDA graph) -> one D2H copy of the step's "
+                         "outputs into pinned host memory (copy stream 2); two device buffer pairs, so "
+                         "step k's copies overlap the compute of steps k - 1 and k + 1; timed from "
+                         "before the first H2D to after the last D2H"),
+                "serial_gbs": round(step_bytes * world * args.steps / t_e2e / 1e9, 2),
+                "serial_path": ("H2D of the step's inputs, the layer calls, D2H of its outputs, all in one "
+                                "CUDA graph per step, one step after another"),
                 "per_layer_copies_gbs": round(step_bytes * world * args.steps / t_e2e_layer / 1e9, 2),
                 "per_layer_copies_path": "H2D of x, the layer call, D2H of y, around every layer call"},
         "gpu_launches": (1 if fused else 2) * n_launch * args.steps,
         "clocks": clocks,
     }
-    del g_step, g_gemm, g_quant, g_two, g_e2e, g_e2e_layer
+    del g_step, g_gemm, g_quant, g_two, g_e2e, g_e2e_layer, g_comp
     if not args.no_extras:
         out["extra"] = extras(args, layers, kernel, peaks, peak_src, world,
                               sm_mhz=(clocks or {}).get("sm_mhz"))
