@@ -451,16 +451,18 @@ __device__ __forceinline__ void fused_activations(const Params& p, int8_t* qbuf,
         int8_t* qr = qbuf + m * QK;
         float4 v[NV];
         float mx = 0.0f;
+        // slots this thread holds (words tid, tid + nthr, ...); the same for
+        // every lane of a warp except in a row's last, partial warp, so the
+        // slots past the row are branched over rather than issued
+        const int nsl = tid < K4 ? (K4 - 1 - tid) / nthr + 1 : 0;
         if constexpr (in_regs) {
-            // predicated loads, all in flight at once; slots past the row
-            // hold zeros, which leave the maximum unchanged
+            // all loads in flight at once
 #pragma unroll
-            for (int u = 0; u < XV; ++u) {
-                const int idx = tid + u * nthr;
-                v[u] = idx < K4 ? xr[idx] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            }
+            for (int u = 0; u < XV; ++u)
+                if (u < nsl) v[u] = xr[tid + u * nthr];
 #pragma unroll
-            for (int u = 0; u < XV; ++u) mx = fmaxf(mx, quant::absmax4(v[u]));
+            for (int u = 0; u < XV; ++u)
+                if (u < nsl) mx = fmaxf(mx, quant::absmax4(v[u]));
         } else {
 #pragma unroll 4
             for (int i = tid; i < K4; i += nthr) mx = fmaxf(mx, quant::absmax4(xr[i]));
@@ -486,7 +488,7 @@ __device__ __forceinline__ void fused_activations(const Params& p, int8_t* qbuf,
 #pragma unroll
             for (int u = 0; u < XV; ++u) {
                 const int idx = tid + u * nthr;
-                if (idx < K4) {
+                if (u < nsl) {
                     const uint32_t w = quant::quantise4(v[u], sc);
                     *reinterpret_cast<uint32_t*>(qr + (idx >> 5) * S + 4 * (idx & 31)) = w;
                     if (qo) qo[idx] = w;
@@ -511,7 +513,6 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     extern __shared__ __align__(16) uint8_t smem[];
     const int M = (int)p.M;
     const int tid = threadIdx.x, nthr = blockDim.x;
-    const int lane = tid & 31, warp = tid >> 5;
     const int64_t r0 = row_begin(p.N, blockIdx.x, p.G), r1 = row_begin(p.N, blockIdx.x + 1, p.G);
     const int Rc = (int)(r1 - r0);
     const int R = p.R, P = p.P, S = p.S, NS = p.NS, CPT = p.CPT;
