@@ -108,11 +108,14 @@ struct Cfg {
     // only while the waiter is not a whole phase ahead of the barrier: a wait
     // for phase k on a barrier still in phase k-1 sees the parity of phase
     // k-2, complete, and returns at once.
-    //  - full(s): the copies of different stages may land in any order, so
-    //    the group waiting for the fill of iteration i must itself have seen
-    //    the fill of iteration i - kStages: kStages a multiple of kDecGroups
-    //    makes it the same group.  It cannot be two phases behind either: the
-    //    next refill of stage s needs this group's arrival on empty(s).
+    //  - code(s) (the stage's codes; the decoders wait for it): the copies of
+    //    different stages may land in any order, so the group waiting for the
+    //    fill of iteration i must itself have seen the fill of iteration
+    //    i - kStages: kStages a multiple of kDecGroups makes it the same
+    //    group.  It cannot be two phases behind either: the next refill of
+    //    stage s needs this group's arrival on empty(s).
+    //  - full(s) (the stage's activation boxes): waited for by the MMA warp
+    //    alone, in stage order; its refill needs the MMA's commit on empty(s).
     //  - aempty(a): completed by tcgen05.commit of the one MMA thread, in
     //    issue order; a group that saw its previous slot freed has seen every
     //    earlier MMA complete, which covers slot a's previous use once the
@@ -123,7 +126,7 @@ struct Cfg {
     // shared memory: [B stages][code stages][barriers + misc]
     static constexpr int kOffCodes = kStages * kBStageBytes;
     static constexpr int kOffBars = kOffCodes + kStages * kCodeStageBytes;
-    static constexpr int kNumBars = 2 * kStages + 2 * kAStages + 2 * kDBufs + 1;
+    static constexpr int kNumBars = 3 * kStages + 2 * kAStages + 2 * kDBufs + 1;
     static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
     static constexpr int kMiscBytes = 64 + 2 * BN * 4;   // tmem holder, flags, token scales [2][BN]
     // output staging for TMA stores: per epilogue warp two slices of
@@ -279,6 +282,10 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
     auto dfull_bar = [&](int d) { return bar0 + 8u * (2 * C::kStages + 2 * C::kAStages + d); };
     auto dempty_bar = [&](int d) { return bar0 + 8u * (2 * C::kStages + 2 * C::kAStages + C::kDBufs + d); };
     const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 2 * C::kAStages + 2 * C::kDBufs);
+    // a stage's codes land on code(s) (the decoders wait for it), its
+    // activation boxes on full(s) (the MMA warp waits for it): the codes of
+    // the first ring round are copied, and decoded, before the dependency wait
+    auto code_bar = [&](int s) { return bar0 + 8u * (2 * C::kStages + 2 * C::kAStages + 2 * C::kDBufs + 1 + s); };
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
@@ -305,6 +312,7 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
     if (threadIdx.x == 32) {
         for (int s = 0; s < C::kStages; ++s) {
             ptx::mbar_init(full_bar(s), 1);
+            ptx::mbar_init(code_bar(s), 1);
             ptx::mbar_init(empty_bar(s), 4 + 1);
         }
         for (int a = 0; a < C::kAStages; ++a) {
@@ -344,9 +352,9 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
         // late delays every role after it.
         //
         // The codes do not depend on the previous kernel: the first ring
-        // round's code copies (each with its stage's whole byte count) are
-        // issued before the dependency wait, so that they overlap the end of
-        // the previous kernel; their activation boxes follow after the wait.
+        // round's code copies are issued before the dependency wait, so that
+        // they (and their decoding) overlap the end of the previous kernel;
+        // their activation boxes follow after the wait.
         int64_t npre = 0;
         {
             SegWalk w(p, blockIdx.x, G);
@@ -357,11 +365,10 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
                 while (left > 0 && npre < C::kStages) {
                     const int nch = left < SC ? left : SC;
                     const uint32_t st = (uint32_t)npre;          // first round: slot npre, no wait
-                    ptx::mbar_arrive_expect_tx_elect(full_bar((int)st),
-                                                     (uint32_t)(nch * (C::kChunkWBytes + C::kBChunkBytes)));
+                    ptx::mbar_arrive_expect_tx_elect(code_bar((int)st), (uint32_t)(nch * C::kChunkWBytes));
                     ptx::bulk_g2s_elect(sbase + C::kOffCodes + st * C::kCodeStageBytes,
                                         p.wnative + (tn * p.Kc + c) * (int64_t)C::kChunkWBytes,
-                                        (uint32_t)(nch * C::kChunkWBytes), full_bar((int)st));
+                                        (uint32_t)(nch * C::kChunkWBytes), code_bar((int)st));
                     c += nch;
                     left -= nch;
                     ++npre;
@@ -393,11 +400,11 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
                 const uint32_t ph1 = (s + 1 == C::kStages) ? ph ^ 1u : ph;
                 const uint32_t t_e = ptx::mbar_test(empty_bar(s1), ph1 ^ 1u);
                 if (!pre) {
-                    ptx::mbar_arrive_expect_tx_elect(full_bar(s),
-                                                     (uint32_t)(nch * (C::kChunkWBytes + C::kBChunkBytes)));
+                    ptx::mbar_arrive_expect_tx_elect(code_bar(s), (uint32_t)(nch * C::kChunkWBytes));
                     ptx::bulk_g2s_elect(sbase + C::kOffCodes + (uint32_t)s * C::kCodeStageBytes, src,
-                                        (uint32_t)(nch * C::kChunkWBytes), full_bar(s));
+                                        (uint32_t)(nch * C::kChunkWBytes), code_bar(s));
                 }
+                ptx::mbar_arrive_expect_tx_elect(full_bar(s), (uint32_t)(nch * C::kBChunkBytes));
                 if (nch == SC) {
 #pragma unroll
                     for (int j = 0; j < SC; ++j)
@@ -426,7 +433,8 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
         int ds = (int)(from % C::kStages);
         uint32_t dph = (uint32_t)((from / C::kStages) & 1);
         for (int64_t i = from; i < issued; ++i) {
-            const bool landed = ptx::mbar_wait_bounded(full_bar(ds), dph, kWaitLimitNs);
+            const bool landed = ptx::mbar_wait_bounded(full_bar(ds), dph, kWaitLimitNs) &&
+                                ptx::mbar_wait_bounded(code_bar(ds), dph, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, landed)) {
                 if (lane == 0) atomicCAS(p.status, 0u, (unsigned)SHERRY_DEV_TIMEOUT_DRAIN);
                 break;
@@ -530,7 +538,7 @@ __global__ void __launch_bounds__(Cfg<BN, SC, WF>::kThreads, 1)
             if (mine) {
                 // no per-stage abort poll: after another role gave up, this
                 // wait runs out by itself and the group leaves
-                bool ok = ptx::mbar_wait_bounded(full_bar(s), sph, kWaitLimitNs);
+                bool ok = ptx::mbar_wait_bounded(code_bar(s), sph, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     if (lane == 0) report(p.status, abort_flag, SHERRY_DEV_TIMEOUT_DECODER);
                     quit = true;
