@@ -182,26 +182,42 @@ __device__ __forceinline__ uint32_t code_x4(const uint32_t (&w)[SHERRY_CHUNK_WOR
     return v & 0x7Cu;
 }
 
+// The decode table: in a static shared array (ST: a lookup is one load at
+// code * 4 plus the array's constant offset) or at a 128-byte aligned
+// address of the dynamic window (a lookup address is (code * 4) | table).
+// Which one measures faster depends on the instantiation (the one-row
+// fused loop keeps the dynamic form).
+struct TableRef {
+    uint32_t addr;              // dynamic form: shared address
+    const uint32_t* ptr;        // static form
+};
+template <bool ST>
+__device__ __forceinline__ uint32_t table_at(const TableRef& t, uint32_t code_x4)
+{
+    if constexpr (ST) return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(t.ptr) + code_x4);
+    else return ptx::lds_u32_nv(code_x4 | t.addr);
+}
+
 // The 4 groups of piece G4 (groups 4 G4 .. 4 G4 + 3) of RT rows: table entries.
-template <int G4, int RT>
-__device__ __forceinline__ void lookup_piece(const uint32_t (&w)[RT][SHERRY_CHUNK_WORDS + 1], uint32_t table_s,
+template <int G4, int RT, bool ST>
+__device__ __forceinline__ void lookup_piece(const uint32_t (&w)[RT][SHERRY_CHUNK_WORDS + 1], const TableRef& tab,
                                              uint32_t (&e)[RT][4])
 {
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
-        e[r][0] = ptx::lds_u32_nv(code_x4<4 * G4 + 0>(w[r]) | table_s);
-        e[r][1] = ptx::lds_u32_nv(code_x4<4 * G4 + 1>(w[r]) | table_s);
-        e[r][2] = ptx::lds_u32_nv(code_x4<4 * G4 + 2>(w[r]) | table_s);
-        e[r][3] = ptx::lds_u32_nv(code_x4<4 * G4 + 3>(w[r]) | table_s);
+        e[r][0] = table_at<ST>(tab, code_x4<4 * G4 + 0>(w[r]));
+        e[r][1] = table_at<ST>(tab, code_x4<4 * G4 + 1>(w[r]));
+        e[r][2] = table_at<ST>(tab, code_x4<4 * G4 + 2>(w[r]));
+        e[r][3] = table_at<ST>(tab, code_x4<4 * G4 + 3>(w[r]));
     }
 }
 
-template <int G4, int MT, int RT>
-__device__ __forceinline__ void piece(const uint32_t (&w)[RT][SHERRY_CHUNK_WORDS + 1], uint32_t table_s,
+template <int G4, int MT, int RT, bool ST>
+__device__ __forceinline__ void piece(const uint32_t (&w)[RT][SHERRY_CHUNK_WORDS + 1], const TableRef& tab,
                                       uint32_t qc, int QK, int M, int32_t (&acc)[RT][MT])
 {
     uint32_t e[RT][4];
-    lookup_piece<G4, RT>(w, table_s, e);
+    lookup_piece<G4, RT, ST>(w, tab, e);
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
         if (m >= M) break;
@@ -550,10 +566,17 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
         else if (busy) fetch_own<RT>(p, r0, Rc, qi * RT, part, k, codes_s + (uint32_t)k * slot_bytes);
         cp_async_commit();
     }
-    // the decode table at a 128-byte aligned shared address, so that a lookup
-    // address is one LOP3: (code * 4) | table
-    const uint32_t table_s = (s_base + kOffTable + 127u) & ~127u;
-    if (tid < 32) ptx::sts_u32(table_s + 4u * (uint32_t)tid, expand_code((uint32_t)tid));
+    // the decode table (see TableRef): static for every instantiation but the
+    // fused one-row one, which measured faster with the dynamic form
+    constexpr bool kStaticTable = !(FUSED && RT == 1);
+    __shared__ __align__(128) uint32_t s_table[32];
+    TableRef tab;
+    tab.addr = (s_base + kOffTable + 127u) & ~127u;
+    tab.ptr = s_table;
+    if (tid < 32) {
+        if constexpr (kStaticTable) s_table[tid] = expand_code((uint32_t)tid);
+        else ptx::sts_u32(tab.addr + 4u * (uint32_t)tid, expand_code((uint32_t)tid));
+    }
     ptx::pdl_wait();
 
     // ---- activations -------------------------------------------------------------
@@ -639,7 +662,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
                     else if (off == 1) v = w[wi] << 1;
                     else if (off <= 27) v = w[wi] >> (off - 2);
                     else v = __funnelshift_r(w[wi], w[wi + 1], off - 2);
-                    e[g] = ptx::lds_u32_nv((v & 0x7Cu) | table_s);
+                    e[g] = table_at<kStaticTable>(tab, v & 0x7Cu);
                 }
                 const uint32_t qc = q_s + (uint32_t)((part * CPT + k) * S);
 #pragma unroll
@@ -683,14 +706,14 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
 #pragma unroll
             for (int r = 0; r < RT; ++r) w[r][SHERRY_CHUNK_WORDS] = 0;
             const uint32_t qc = q_s + (uint32_t)(c * S);
-            piece<0, MT, RT>(w, table_s, qc, QK, M, acc);
-            piece<1, MT, RT>(w, table_s, qc, QK, M, acc);
-            piece<2, MT, RT>(w, table_s, qc, QK, M, acc);
-            piece<3, MT, RT>(w, table_s, qc, QK, M, acc);
-            piece<4, MT, RT>(w, table_s, qc, QK, M, acc);
-            piece<5, MT, RT>(w, table_s, qc, QK, M, acc);
-            piece<6, MT, RT>(w, table_s, qc, QK, M, acc);
-            piece<7, MT, RT>(w, table_s, qc, QK, M, acc);
+            piece<0, MT, RT, kStaticTable>(w, tab, qc, QK, M, acc);
+            piece<1, MT, RT, kStaticTable>(w, tab, qc, QK, M, acc);
+            piece<2, MT, RT, kStaticTable>(w, tab, qc, QK, M, acc);
+            piece<3, MT, RT, kStaticTable>(w, tab, qc, QK, M, acc);
+            piece<4, MT, RT, kStaticTable>(w, tab, qc, QK, M, acc);
+            piece<5, MT, RT, kStaticTable>(w, tab, qc, QK, M, acc);
+            piece<6, MT, RT, kStaticTable>(w, tab, qc, QK, M, acc);
+            piece<7, MT, RT, kStaticTable>(w, tab, qc, QK, M, acc);
         }
         if (streaming && k + NS < CPT) {
             if (own) {
