@@ -34,8 +34,12 @@
 //
 // Warp roles (576 threads; 448 for 192-token tiles with two-chunk stages,
 // which have two decoder groups):
-//   warp 0       producer: per stage one bulk copy of the codes and one 2D
-//                TMA of the activation tile per chunk
+//   warp 0       producer: per stage one bulk copy of the codes (completing
+//                the stage's code barrier, which the decoders wait for) and
+//                one 2D TMA of the activation tile per chunk (completing its
+//                full barrier, which the MMA warp waits for); the codes of
+//                the first ring round go out before the dependency wait, so
+//                the decoders work while the previous kernel finishes
 //   warp 1       TMEM allocation and MMA issue (an elected lane)
 //   warps 2-13   three decoder groups of four warps (each group covers the
 //                four TMEM lane quadrants), taking stages in turn
