@@ -145,3 +145,95 @@ def test_a_ring_at_least_as_deep_as_the_groups_is_safe(A, G):
 @pytest.mark.parametrize("A,G", [(2, 3), (1, 2)])
 def test_a_ring_shallower_than_the_groups_is_not(A, G):
     assert any(run_a_ring(A, G, 60, seed) > 0 for seed in range(400))
+
+
+def run_split_ring(S: int, G: int, iters: int, seed: int, pre: int) -> int:
+    """The stage ring with a stage's codes and activations on separate
+    barriers: code(s) completes when the codes land (decoder group g parity-
+    waits on it for its iterations i = g mod G), full(s) when the activation
+    boxes land (the MMA parity-waits on it, in order, after the decoders'
+    hand-off).  The two copies of a fill land independently, in any order
+    across stages.  The codes of the first `pre` iterations are issued before
+    anything else may move (before the dependency wait); their activation
+    boxes, and every later fill, only once empty(s) saw both the decoders'
+    and the MMA's arrivals for the stage's previous round.  Returns the
+    number of stale reads (a waiter passing while the stage holds another
+    iteration's codes or activations); 1000 more if the model gets stuck."""
+    rng = random.Random(seed)
+    code_done = [0] * S
+    act_done = [0] * S
+    code_tag = [-1] * S
+    act_tag = [-1] * S
+    dec_arr = [0] * S
+    mma_arr = [0] * S
+    in_code, in_act = [], []
+    next_code = min(pre, S, iters)      # codes already issued before the wait
+    in_code.extend(range(next_code))
+    next_act = 0
+    dec_next = list(range(G))
+    dec_done = [False] * iters
+    mma_next = 0
+    bad = 0
+
+    def passes(done: int, k: int) -> bool:
+        return (done & 1) != (k & 1)
+
+    while mma_next < iters:
+        moves = []
+        # a fill (codes + activations, or activations alone for a pre-issued
+        # iteration) once the stage's previous round is released
+        j = next_act
+        if j < iters and min(dec_arr[j % S], mma_arr[j % S]) >= j // S:
+            moves.append("fill")
+        if in_code:
+            moves.append("land_code")
+        if in_act:
+            moves.append("land_act")
+        for g in range(G):
+            i = dec_next[g]
+            if i < iters and passes(code_done[i % S], i // S):
+                moves.append(("dec", g))
+        if mma_next < iters and dec_done[mma_next] and passes(act_done[mma_next % S], mma_next // S):
+            moves.append("mma")
+        if not moves:
+            return bad + 1000
+        mv = rng.choice(moves)
+        if mv == "fill":
+            if j >= next_code:
+                in_code.append(j)
+                next_code = j + 1
+            in_act.append(j)
+            next_act += 1
+        elif mv == "land_code":
+            c = in_code.pop(rng.randrange(len(in_code)))
+            code_tag[c % S] = c
+            code_done[c % S] += 1
+        elif mv == "land_act":
+            a = in_act.pop(rng.randrange(len(in_act)))
+            act_tag[a % S] = a
+            act_done[a % S] += 1
+        elif mv == "mma":
+            if act_tag[mma_next % S] != mma_next:
+                bad += 1
+            mma_arr[mma_next % S] += 1
+            mma_next += 1
+        else:
+            g = mv[1]
+            i = dec_next[g]
+            if code_tag[i % S] != i:
+                bad += 1
+            dec_done[i] = True
+            dec_arr[i % S] += 1
+            dec_next[g] += G
+    return bad
+
+
+@pytest.mark.parametrize("S,G", [(3, 3), (6, 3), (9, 3), (2, 2), (4, 2), (6, 2)])
+@pytest.mark.parametrize("pre", [0, 1, 100])
+def test_split_barrier_rings_never_read_a_stale_stage(S, G, pre):
+    assert all(run_split_ring(S, G, 60, seed, pre) == 0 for seed in range(300))
+
+
+@pytest.mark.parametrize("S,G", [(4, 3), (5, 3), (7, 3)])
+def test_split_barrier_rings_off_whole_rounds_can(S, G):
+    assert any(run_split_ring(S, G, 60, seed, 100) > 0 for seed in range(400))
